@@ -1,0 +1,211 @@
+"""Pins of the oracle's quantizers (1x16, 16x16, transposed, RHT, SR forms).
+
+gist.science "Pretraining Large Language Models with NVFP4", Technische Zusammenfassung:
+2.A -- 16-element blocks, E4M3 block scales, an FP32 tensor-level scale, "about 6.25 % of the
+values in a block encoded at near FP8 precision" (the block's largest element); 2.B.3 -- 16x16
+weight blocks make the quantized weight identical in forward and backward (transposed).
+"""
+import os
+
+import numpy as np
+import pytest
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_blocks.txt")
+
+
+def _golden():
+    out = {}
+    for line in open(GOLDEN):
+        if line.startswith("#") or ":" not in line:
+            continue
+        k, v = line.split(":", 1)
+        out[k.strip()] = [int(t, 16) for t in v.split()]
+    return out
+
+
+def test_hand_worked_blocks(ora):
+    g = _golden()
+    x = np.array(g["x_bf16"], np.uint16).reshape(1, 48)
+    q = ora.quantize(x)
+    assert q.amax == 6.0
+    assert q.s_t == np.float32(6.0) / np.float32(2688.0)
+    assert q.codes.reshape(-1).tolist() == g["codes"]
+    assert q.scales_rm.reshape(-1).tolist() == g["scales"]
+    assert q.scales_sw[:3].tolist() == g["scales"] and not q.scales_sw[3:].any()
+
+
+def test_hand_worked_16x16_tile(ora):
+    # one 16x16 weight tile: W[0][0] = 6, every other entry 0.5.  One scale for the tile:
+    # amax 6 -> S_enc 448, s_b = 448 (0x7E), codes 7 and 1 (0.5 exactly).  A 1x16 row block
+    # would instead give rows 1..15 their own scale from amax 0.5.
+    w = np.full((16, 16), 0.5, np.float32)
+    w[0, 0] = 6.0
+    bits = (w.view(np.uint32) >> 16).astype(np.uint16)
+    q = ora.quantize(bits, block=ora.BLOCK_16x16)
+    assert q.tile_scales.tolist() == [[0x7E]]
+    assert np.all(q.scales_rm == 0x7E)
+    nib = q.nibbles()
+    assert nib[0, 0] == 7 and np.all(nib.reshape(-1)[1:] == 1)
+    q1 = ora.quantize(bits, block=ora.BLOCK_1x16)
+    assert q1.scales_rm[0, 0] == 0x7E and np.all(q1.scales_rm[1:, 0] == ora.e4m3_rne_sat(
+        np.array([np.float32(np.float32(0.5) / np.float32(6.0)) * np.float32(448.0)]))[0])
+
+
+def _x(rows, cols, seed=0, outliers=0.0):
+    return synth.bf16_bits(synth.activations(rows, cols, seed=seed, outlier_frac=outliers))
+
+
+@pytest.mark.parametrize("along,mode,block,rht", [
+    (0, 0, 0, False), (1, 0, 0, True), (0, 1, 0, False), (1, 1, 0, True), (0, 0, 1, False), (1, 0, 0, False)])
+def test_amax_element_maps_to_six(ora, along, mode, block, rht):
+    x = _x(256, 512, seed=3, outliers=0.01)
+    q = ora.quantize(x, along=along, mode=mode, block=block, rht=rht, rht_seed=5, sr_seed=9, stream_id=1)
+    v = _form_values(ora, x, along, rht, 5)
+    R, K = v.shape
+    nib = q.nibbles()
+    sc = q.scales_rm
+    normal = (sc >= 0x08) & (sc < 0x7E)   # normal E4M3 scales below 448
+    checked = 0
+    for r in range(R):
+        for kb in range(K // 16):
+            if not normal[r, kb]:
+                continue
+            if block == 0:
+                blk = np.abs(v[r, kb * 16:(kb + 1) * 16])
+                j = int(np.argmax(blk))
+                # u of the block maximum lies in [6/(1+2^-4), 6/(1-2^-4)] = [5.65, 6.4]: RNE gives
+                # 6; SR gives 6 or its lower neighbour 4
+                assert nib[r, kb * 16 + j] & 7 in ((7,) if mode == 0 else (6, 7))
+            checked += 1
+    assert checked > 0
+    # the block holding the tensor amax gets the largest scale, 448
+    assert sc.max() == 0x7E
+
+
+def _form_values(ora, x_bits, along, rht, rht_seed):
+    v = ora.bf16_bits_to_f32(x_bits).reshape(x_bits.shape)
+    if along:
+        v = v.T.copy()
+    if rht:
+        signs = ora.rht_signs(rht_seed)
+        R, K = v.shape
+        v = np.stack([np.concatenate([ora.rht16(v[r, k:k + 16], signs) for k in range(0, K, 16)]) for r in range(R)])
+    return v.astype(np.float32)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_reconstruction_bound(ora, mode):
+    # x_hat = q * dec(s_b) * s_t.  Per element |x - x_hat| <= (half an E2M1 step for RNE, one
+    # step for SR) * dec(s_b) * S_dec, except above the grid (saturation); blocks are checked
+    # only where the scale is normal.
+    x = _x(128, 1024, seed=11, outliers=0.005)
+    q = ora.quantize(x, mode=mode, sr_seed=3, stream_id=1)
+    v = ora.bf16_bits_to_f32(x).reshape(x.shape).astype(np.float64)
+    xh = q.dequantize()
+    s_enc = np.float64(np.float32(2688.0) / np.float32(q.amax))
+    dec = np.array([ora.e4m3_value(c) for c in range(256)])[q.scales_rm].repeat(16, axis=1)
+    unit = dec / s_enc                 # value of one E2M1 unit in x's scale (approximately)
+    u = np.abs(v) / np.where(unit > 0, unit, 1)
+    steps = np.select([u < 2, u < 4], [0.5, 1.0], 2.0)
+    factor = 0.5 if mode == 0 else 1.0
+    ok = (q.scales_rm.repeat(16, axis=1) >= 0x08) & (u <= 6.0)
+    err = np.abs(v - xh)
+    bound = factor * steps * unit * (1 + 1e-6) + 1e-30
+    assert np.all(err[ok] <= bound[ok])
+
+
+def test_16x16_transpose_identity(ora):
+    w = synth.bf16_bits(synth.weights(96, 160, seed=1))
+    q = ora.quantize(w, block=ora.BLOCK_16x16)
+    qt = ora.transpose_2d(q)
+    qT = ora.quantize(np.ascontiguousarray(w.T), block=ora.BLOCK_16x16)
+    assert np.array_equal(qt.codes, qT.codes)
+    assert np.array_equal(qt.scales_rm, qT.scales_rm)
+    assert np.array_equal(qt.scales_sw, qT.scales_sw)
+    assert np.array_equal(qt.tile_scales, qT.tile_scales)
+    assert qt.s_t == qT.s_t
+    # dequantized transposed weight equals the transposed dequantized weight, bit for bit
+    assert np.array_equal(qt.dequantize(), q.dequantize().T)
+    # the along=1 form of a 16x16 quantization is the transpose as well
+    q1 = ora.quantize(w, along=1, block=ora.BLOCK_16x16)
+    assert np.array_equal(q1.codes, qt.codes) and np.array_equal(q1.scales_rm, qt.scales_rm)
+
+
+def test_along1_equals_transposed_input(ora):
+    x = _x(64, 96, seed=4)
+    for rht in (False, True):
+        a = ora.quantize(x, along=1, rht=rht, rht_seed=17)
+        b = ora.quantize(np.ascontiguousarray(x.T), along=0, rht=rht, rht_seed=17)
+        assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales_sw, b.scales_sw)
+        assert a.s_t == b.s_t
+
+
+def test_rht_amax_is_over_transformed_values(ora):
+    x = _x(64, 48, seed=8, outliers=0.05)
+    q = ora.quantize(x, along=1, rht=True, rht_seed=2)
+    v = _form_values(ora, x, 1, True, 2)
+    assert q.amax == np.abs(v).max()
+    assert q.amax != np.abs(ora.bf16_bits_to_f32(x)).max()
+
+
+def test_swizzle_layout_is_a_padded_permutation(ora):
+    for R, K in ((128, 64), (200, 48), (256, 512), (1, 16), (130, 80)):
+        n = ora.scales_sw_bytes(R, K)
+        seen = np.zeros(n, bool)
+        for r in range(R):
+            for kb in range(K // 16):
+                o = ora.swizzle_offset(r, kb, K)
+                assert 0 <= o < n and not seen[o]
+                seen[o] = True
+        assert seen.sum() == R * (K // 16)
+    # the four scales of one row inside one 64-element K tile are adjacent bytes
+    assert [ora.swizzle_offset(5, kb, 256) for kb in range(4)] == [80, 81, 82, 83]
+    # rows 32 apart share a 16-byte line
+    assert ora.swizzle_offset(37, 0, 256) == ora.swizzle_offset(5, 0, 256) + 4
+
+
+def test_sr_reproducible_and_seed_dependent(ora):
+    dy = synth.bf16_bits(synth.grad_output(64, 256, seed=2))
+    a = ora.quantize(dy, mode=ora.SR, sr_seed=5, stream_id=1)
+    b = ora.quantize(dy, mode=ora.SR, sr_seed=5, stream_id=1)
+    c = ora.quantize(dy, mode=ora.SR, sr_seed=6, stream_id=1)
+    rne = ora.quantize(dy, mode=ora.RNE)
+    assert np.array_equal(a.codes, b.codes)
+    assert np.array_equal(a.scales_rm, rne.scales_rm)     # scales always use RNE
+    diff = np.mean(a.nibbles() != c.nibbles())
+    assert 0.2 < diff < 0.8
+
+
+def test_zero_tensor_and_empty(ora):
+    z = np.zeros((32, 64), np.uint16)
+    q = ora.quantize(z)
+    assert q.amax == 0.0 and q.s_t == 1.0
+    assert not q.codes.any() and not q.scales_rm.any()
+    neg = np.full((16, 16), 0x8000, np.uint16)   # -0.0
+    assert np.all(ora.quantize(neg).nibbles() == 8)
+    e = ora.quantize(np.zeros((0, 32), np.uint16))
+    assert e.codes.size == 0 and e.s_t == 1.0
+
+
+def test_nonfinite_rejected(ora):
+    x = np.zeros((16, 16), np.uint16)
+    x[3, 4] = 0x7F80   # +inf
+    with pytest.raises(ValueError):
+        ora.quantize(x)
+    x[3, 4] = 0x7FC1   # NaN
+    with pytest.raises(ValueError):
+        ora.quantize(x)
+
+
+def test_threads_bit_identical(ora):
+    x = _x(200, 320, seed=21)
+    for kw in (dict(), dict(along=1, rht=True, mode=1, sr_seed=4, stream_id=2), dict(block=1, along=0)):
+        if kw.get("block") == 1:
+            x2 = x[:192]
+        else:
+            x2 = x[:192] if kw.get("along") else x
+        a = ora.quantize(x2, nthreads=1, **kw)
+        b = ora.quantize(x2, nthreads=7, **kw)
+        assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales_sw, b.scales_sw)
