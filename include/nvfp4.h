@@ -1,0 +1,208 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4: NVFP4 quantization fused into block-scaled FP4 GEMMs for the
+ * fprop, dgrad and wgrad GEMMs of a linear layer, on one B200 (sm_100a).
+ *
+ * What the operations are follows the pages on NVIDIA's report "Pretraining Large Language
+ * Models with NVFP4" (gist.science, Technische Zusammenfassung 2.A and 2.B; webconsulting.at,
+ * "Das Wichtigste"; brainai.pro, "Details techniques"):
+ *   - NVFP4 = 4-bit E2M1 elements, one E4M3 scale per 16 consecutive elements, one FP32 scale
+ *     per tensor (2.A "Das NVFP4-Format");
+ *   - weights use 16x16 2D blocks so forward and backward see the same quantized weight
+ *     (2.B.3);
+ *   - a seeded 16-point Random Hadamard Transform is applied along K to both Wgrad operands
+ *     only (2.B.2);
+ *   - gradients are rounded stochastically, activations and weights round-to-nearest-even
+ *     (2.B.4);
+ *   - the GEMMs run on the Blackwell FP4 tensor cores (3, "Hardware-Nutzung").
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are caller-owned DEVICE pointers.  The library never allocates,
+ *     never frees, never prints and never throws across this boundary.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and returns after validating its arguments and enqueuing its kernels.  Argument checks
+ *     are synchronous and happen before any launch: a non-OK status means nothing was enqueued
+ *     (except NVFP4_ERR_CUDA, which reports a failed launch; the CUDA error is consumed).
+ *   - Conditions detected on the device (NaN/Inf input, a device-side wait that ran out of its
+ *     time budget) set flags in the caller's workspace; read them with nvfp4_poll().
+ *   - Layouts: bf16 inputs are row-major with a leading dimension in elements.  A quantized
+ *     form (nvfp4_tensor) has `rows` rows and `k` elements along the GEMM reduction axis:
+ *       codes        [rows][k/2] bytes, K-major, element 2j in the low nibble of byte j;
+ *       scales       E4M3 block scales in 128x4 tiles of 512 bytes: the scale of (row r,
+ *                    block kb = k_index/16) sits at ((r/128)*ceil(k/64) + kb/4)*512
+ *                    + (r%32)*16 + ((r/32)%4)*4 + kb%4; padding bytes are zero (this is the
+ *                    layout the tcgen05 block-scaled MMA reads through tcgen05.cp);
+ *       tile_scales  16x16 forms only: compact grid [rows/16][k/16] (may be NULL);
+ *       tensor_scale one fp32: the decode scale s_t = amax_t / (6*448).
+ *     A value is reconstructed as e2m1(code) * e4m3(scale) * s_t.
+ *   - Alignment: every device pointer 16-byte aligned.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = 1,        /* a required pointer is NULL */
+    NVFP4_ERR_ALIGN = 2,       /* a pointer or leading dimension breaks the 16-byte rule */
+    NVFP4_ERR_SHAPE = 3,       /* a size violates the operation's shape rule (see each call) */
+    NVFP4_ERR_ARG = 4,         /* an enum or flag out of range, or inconsistent operands */
+    NVFP4_ERR_WORKSPACE = 5,   /* workspace NULL */
+    NVFP4_ERR_CUDA = 6,        /* a CUDA launch or runtime call failed */
+    NVFP4_ERR_NONFINITE = 7,   /* (nvfp4_poll) NaN or Inf seen by an amax pass */
+    NVFP4_ERR_TIMEOUT = 8,     /* (nvfp4_poll) a device-side wait ran out of its time budget */
+    NVFP4_ERR_UNSUPPORTED = 9, /* the device is not sm_100 */
+    NVFP4_ERR_LIMIT = 10       /* a size exceeds a fixed limit of the call */
+} nvfp4_status;
+
+typedef enum { NVFP4_RNE = 0, NVFP4_SR = 1 } nvfp4_round;
+typedef enum { NVFP4_BLOCK_1x16 = 0, NVFP4_BLOCK_16x16 = 1 } nvfp4_block;
+typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_FP32 = 1 } nvfp4_dtype;
+
+/* Philox stream ids used by the linear layer (the counter's third word). */
+#define NVFP4_STREAM_DGRAD 1u   /* dY, 1x16 along the output features (dgrad operand) */
+#define NVFP4_STREAM_WGRAD 2u   /* dY^T after the RHT, 1x16 along tokens (wgrad operand) */
+#define NVFP4_STREAM_RHT 3u     /* reserved: the RHT sign draw */
+
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    uint8_t* tile_scales;
+    float* tensor_scale;
+    int64_t rows;
+    int64_t k;
+    int32_t block;     /* nvfp4_block */
+    int32_t reserved;
+} nvfp4_tensor;
+
+/* ---- sizes (host, pure functions) ------------------------------------------------------ */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t k);       /* rows * k / 2 */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t k);      /* ceil(rows/128)*128 * ceil(k/64)*4 */
+size_t nvfp4_tile_scales_bytes(int64_t rows, int64_t k); /* (rows/16) * (k/16) */
+size_t nvfp4_workspace_bytes(void);                      /* 256 */
+
+/* Zero a workspace (flags and amax slots).  Call once after allocating it. */
+nvfp4_status nvfp4_workspace_init(void* ws, nvfp4_stream_t stream);
+
+/*
+ * Quantize one operand form of a bf16 tensor x[rows][ldx] (logical width `cols`).
+ * along = 0: the form is x itself (form rows = rows, k = cols).
+ * along = 1: the form is x^T (form rows = cols, k = rows) -- the token-major wgrad operands.
+ * block: 1x16 along k, or 16x16 tiles (weights).  rht = 1 applies the seeded 16-point RHT
+ * along k before anything else (1x16 only).  mode = NVFP4_SR draws one 16-bit Philox field
+ * per element: key = sr_seed, counter = (i/8 lo, i/8 hi, stream_id, 0), i = the element's
+ * row-major index r*cols + c in x.  The RHT signs are bit j of word 0 of
+ * Philox(key = rht_seed, counter = (0, 0, 3, 0)), set = -1.
+ * Two passes over x: an amax reduction (over the transformed values when rht = 1) and the
+ * quantize pass; tensor scales S_enc = 2688/amax_t, s_t = amax_t/2688 (1 and 1 if amax_t == 0).
+ * Shape rules: k % 16 == 0; along = 1 or 16x16 needs form rows % 16 == 0 and k % 16 == 0;
+ * cols % 16 == 0 always.  rows or cols == 0 is a no-op that writes s_t = 1.
+ * out: codes/scales/tensor_scale required, tile_scales required for 16x16 (else ignored);
+ * out->rows/k/block are written by the call.  ws: a workspace of nvfp4_workspace_bytes().
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along,
+                            nvfp4_round mode, nvfp4_block block, int rht, uint64_t rht_seed,
+                            uint64_t sr_seed, uint32_t stream_id, nvfp4_tensor* out, void* ws,
+                            nvfp4_stream_t stream);
+
+/*
+ * One read of x, two forms (gist.science 2.B.2: RHT only for the Wgrad inputs):
+ *   out_row: along = 0, 1x16, no RHT, rounding `mode`, Philox stream `stream_row`
+ *            (fprop operand X, dgrad operand dY);
+ *   out_col: along = 1, 1x16, RHT (rht_seed), rounding `mode`, Philox stream `stream_col`
+ *            (wgrad operands X^T, dY^T).
+ * Results are bit-identical to two nvfp4_quantize calls with the same arguments.
+ * Shape rules: rows % 16 == 0, cols % 16 == 0.
+ */
+nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                 nvfp4_round mode, uint64_t rht_seed, uint64_t sr_seed,
+                                 uint32_t stream_row, uint32_t stream_col, nvfp4_tensor* out_row,
+                                 nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream);
+
+/*
+ * 16x16 weight quantization (gist.science 2.B.3), RNE, writing the forward form w_q
+ * ([rows][cols], k = cols) and, if w_qt is not NULL, the transposed dgrad form
+ * ([cols][rows], k = rows) from the same registers -- bit-identical to nvfp4_transpose_2d of
+ * w_q.  Shape rules: rows % 16 == 0, cols % 16 == 0.  tile_scales of w_q is required.
+ */
+nvfp4_status nvfp4_quantize_weight(const void* w, int64_t rows, int64_t cols, int64_t ldw,
+                                   nvfp4_tensor* w_q, nvfp4_tensor* w_qt, void* ws,
+                                   nvfp4_stream_t stream);
+
+/*
+ * Transposed layout of a 16x16-quantized tensor without requantizing (gist.science 2.B.3):
+ * wt->codes[k][r] = w->codes[r][k], tile grid transposed, same tensor scale (copied).
+ * w->block must be NVFP4_BLOCK_16x16 with tile_scales; wt->tile_scales may be NULL.
+ */
+nvfp4_status nvfp4_transpose_2d(const nvfp4_tensor* w, nvfp4_tensor* wt, nvfp4_stream_t stream);
+
+/*
+ * D[M][N] = s_tA * s_tB * sum_k A[m][k] * B[n][k]: both operands K-major quantized forms with
+ * the same k (brainai.pro "Details techniques": the FP4 GEMMs of the fully connected layers).
+ * M = a->rows, N = b->rows, K = a->k.  fp32 accumulation in tensor memory; bf16 or fp32 output
+ * with leading dimension ldd (elements).  Shape rules: K % 32 == 0 and K > 0; M, N >= 1;
+ * ldd >= N and ldd * sizeof(out) % 16 == 0.  ws receives the timeout flag.
+ */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, int64_t ldd,
+                        nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream);
+
+/*
+ * Linear layer y = x w^T with NVFP4 GEMMs (gist.science 2.B): all buffers caller-owned.
+ *   xq      [T][d]   1x16 RNE           (fprop A)
+ *   xq_rht  [d][T]   RHT 1x16 RNE       (wgrad B)
+ *   wq      [n][d]   16x16 RNE          (fprop B; tile_scales required)
+ *   wqt     [d][n]   16x16 transposed   (dgrad B)
+ *   dyq     [T][n]   1x16 SR stream 1   (dgrad A)
+ *   dyq_rht [n][T]   RHT 1x16 SR stream 2 (wgrad A)
+ * w_cached != 0 makes nvfp4_linear_fwd reuse wq/wqt as they are.  Shape rules: T % 64 == 0,
+ * d % 64 == 0, n % 64 == 0 (each is a K of one GEMM and a 16-row tile dimension).
+ */
+typedef struct {
+    int64_t T, d, n;
+    uint64_t rht_seed;
+    nvfp4_tensor xq, xq_rht, wq, wqt, dyq, dyq_rht;
+    void* ws;
+    int32_t w_cached;
+    int32_t reserved;
+} nvfp4_linear_ctx;
+
+/* Forward: quantize W (16x16, both layouts) unless cached, quantize X (both forms), then
+ * y[T][n] (bf16) = GEMM(xq, wq). */
+nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linear_ctx* ctx,
+                              nvfp4_stream_t stream);
+
+/* Backward: quantize dY (both forms, SR with sr_seed), dx[T][d] (bf16) = GEMM(dyq, wqt),
+ * dw[n][d] (fp32) = GEMM(dyq_rht, xq_rht).  dx or dw may be NULL to skip that GEMM. */
+nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float* dw,
+                              nvfp4_linear_ctx* ctx, nvfp4_stream_t stream);
+
+/* GeLU glue of the one-FFN training step (erf form, fp32 math, bf16 in and out):
+ * g = 0.5 h (1 + erf(h / sqrt 2));  dh = dg * (Phi(h) + h phi(h)).  n elements, contiguous. */
+nvfp4_status nvfp4_gelu_fwd(const void* h, void* g, int64_t n, nvfp4_stream_t stream);
+nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n,
+                            nvfp4_stream_t stream);
+
+/* Synchronize `stream`, then report (and clear) the device flags of `ws`: NVFP4_ERR_TIMEOUT
+ * takes precedence over NVFP4_ERR_NONFINITE; NVFP4_OK when neither is set. */
+nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream);
+
+/* Device-side wait budget of the GEMM's mbarrier spins, in nanoseconds (default 2e9).
+ * Process-wide; 0 restores the default. */
+void nvfp4_set_wait_budget_ns(uint64_t ns);
+
+const char* nvfp4_status_string(nvfp4_status s);
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,313 @@
+"""Python binding of libnvfp4 (include/nvfp4.h): NVFP4 quantization and block-scaled FP4 GEMMs
+for the fprop, dgrad and wgrad GEMMs of a linear layer on a B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libnvfp4.so``.  PyTorch provides device memory and the current stream.  Importing this
+module does not load the library; the first call does, and raises if it is missing -- there is
+no CPU fallback.
+
+The functions carry the C names: ``nvfp4_quantize``, ``nvfp4_quantize_dual``,
+``nvfp4_quantize_weight``, ``nvfp4_transpose_2d``, ``nvfp4_gemm``, ``nvfp4_linear_fwd``,
+``nvfp4_linear_bwd``, ``nvfp4_gelu_fwd``, ``nvfp4_gelu_bwd``, ``nvfp4_poll``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
+
+RNE, SR = 0, 1
+BLOCK_1x16, BLOCK_16x16 = 0, 1
+OUT_BF16, OUT_FP32 = 0, 1
+STREAM_DGRAD, STREAM_WGRAD, STREAM_RHT = 1, 2, 3
+
+STATUS = {0: "OK", 1: "ERR_NULL", 2: "ERR_ALIGN", 3: "ERR_SHAPE", 4: "ERR_ARG", 5: "ERR_WORKSPACE", 6: "ERR_CUDA",
+          7: "ERR_NONFINITE", 8: "ERR_TIMEOUT", 9: "ERR_UNSUPPORTED", 10: "ERR_LIMIT"}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_lib().nvfp4_status_string(status).decode()})")
+
+
+class CTensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("tile_scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("block", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class CLinearCtx(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("n", ctypes.c_int64), ("rht_seed", ctypes.c_uint64),
+                ("xq", CTensor), ("xq_rht", CTensor), ("wq", CTensor), ("wqt", CTensor), ("dyq", CTensor),
+                ("dyq_rht", CTensor), ("ws", ctypes.c_void_p), ("w_cached", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_L = None
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libnvfp4.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        vp, i64, u64, u32, i32 = c.c_void_p, c.c_int64, c.c_uint64, c.c_uint32, c.c_int
+        T = c.POINTER(CTensor)
+        sig = {
+            "nvfp4_codes_bytes": ([i64, i64], c.c_size_t),
+            "nvfp4_scales_bytes": ([i64, i64], c.c_size_t),
+            "nvfp4_tile_scales_bytes": ([i64, i64], c.c_size_t),
+            "nvfp4_workspace_bytes": ([], c.c_size_t),
+            "nvfp4_workspace_init": ([vp, vp], i32),
+            "nvfp4_quantize": ([vp, i64, i64, i64, i32, i32, i32, i32, u64, u64, u32, T, vp, vp], i32),
+            "nvfp4_quantize_dual": ([vp, i64, i64, i64, i32, u64, u64, u32, u32, T, T, vp, vp], i32),
+            "nvfp4_quantize_weight": ([vp, i64, i64, i64, T, T, vp, vp], i32),
+            "nvfp4_transpose_2d": ([T, T, vp], i32),
+            "nvfp4_gemm": ([T, T, vp, i64, i32, vp, vp], i32),
+            "nvfp4_linear_fwd": ([vp, vp, vp, c.POINTER(CLinearCtx), vp], i32),
+            "nvfp4_linear_bwd": ([vp, u64, vp, vp, c.POINTER(CLinearCtx), vp], i32),
+            "nvfp4_gelu_fwd": ([vp, vp, i64, vp], i32),
+            "nvfp4_gelu_bwd": ([vp, vp, vp, i64, vp], i32),
+            "nvfp4_poll": ([vp, vp], i32),
+            "nvfp4_set_wait_budget_ns": ([u64], None),
+            "nvfp4_status_string": ([i32], c.c_char_p),
+            "nvfp4_version": ([], i32),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _L = L
+    return _L
+
+
+def lib():
+    """The loaded ctypes library (raises ImportError if it is not built)."""
+    return _lib()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise NVFP4Error(status, what)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# ---------------------------------------------------------------------------------------
+# workspace
+# ---------------------------------------------------------------------------------------
+class Workspace:
+    """256 bytes of device memory for amax slots and the sticky device flags."""
+
+    def __init__(self, device=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.buf = torch.empty(_lib().nvfp4_workspace_bytes(), dtype=torch.uint8, device=device)
+        _check(_lib().nvfp4_workspace_init(_ptr(self.buf), _stream()), "nvfp4_workspace_init")
+
+    @property
+    def ptr(self):
+        return _ptr(self.buf)
+
+
+_DEFAULT_WS = {}
+
+
+def default_workspace() -> Workspace:
+    dev = torch.cuda.current_device()
+    if dev not in _DEFAULT_WS:
+        _DEFAULT_WS[dev] = Workspace()
+    return _DEFAULT_WS[dev]
+
+
+def nvfp4_poll(ws: Workspace | None = None, stream=None) -> int:
+    """Synchronize the stream and return (and clear) the workspace's device status."""
+    ws = ws or default_workspace()
+    return _lib().nvfp4_poll(ws.ptr, _stream(stream))
+
+
+def nvfp4_set_wait_budget_ns(ns: int):
+    _lib().nvfp4_set_wait_budget_ns(int(ns))
+
+
+# ---------------------------------------------------------------------------------------
+# quantized operand forms
+# ---------------------------------------------------------------------------------------
+@dataclass
+class NVFP4Tensor:
+    """One quantized operand form (device buffers owned by torch)."""
+    codes: torch.Tensor          # uint8 [rows][k/2]
+    scales: torch.Tensor         # uint8, 128x4-tile swizzled E4M3 block scales
+    tile_scales: torch.Tensor | None  # uint8 [rows/16][k/16] for 16x16 forms
+    tensor_scale: torch.Tensor   # float32 [1]: decode scale s_t
+    rows: int
+    k: int
+    block: int
+
+    @staticmethod
+    def empty(rows: int, k: int, block: int = BLOCK_1x16, device=None) -> "NVFP4Tensor":
+        L = _lib()
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        codes = torch.empty(max(L.nvfp4_codes_bytes(rows, k), 1), dtype=torch.uint8, device=device)
+        scales = torch.empty(max(L.nvfp4_scales_bytes(rows, k), 16), dtype=torch.uint8, device=device)
+        tiles = None
+        if block == BLOCK_16x16:
+            tiles = torch.empty(max(L.nvfp4_tile_scales_bytes(rows, k), 1), dtype=torch.uint8, device=device)
+        st = torch.empty(1, dtype=torch.float32, device=device)
+        return NVFP4Tensor(codes, scales, tiles, st, rows, k, block)
+
+    def c(self) -> CTensor:
+        return CTensor(self.codes.data_ptr(), self.scales.data_ptr(),
+                       self.tile_scales.data_ptr() if self.tile_scales is not None else None,
+                       self.tensor_scale.data_ptr(), self.rows, self.k, self.block, 0)
+
+    def codes_2d(self) -> torch.Tensor:
+        return self.codes[: self.rows * (self.k // 2)].view(self.rows, self.k // 2)
+
+
+def _bf16_2d(x: torch.Tensor):
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("expected a 2-D bf16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("inner dimension must be contiguous")
+    return x.shape[0], x.shape[1], x.stride(0)
+
+
+def nvfp4_quantize(x: torch.Tensor, along: int = 0, mode: int = RNE, block: int = BLOCK_1x16, rht: bool = False,
+                   rht_seed: int = 0, sr_seed: int = 0, stream_id: int = 0, out: NVFP4Tensor | None = None,
+                   ws: Workspace | None = None, stream=None) -> NVFP4Tensor:
+    rows, cols, ld = _bf16_2d(x)
+    R, K = (cols, rows) if along else (rows, cols)
+    out = out or NVFP4Tensor.empty(R, K, block, x.device)
+    ws = ws or default_workspace()
+    ct = out.c()
+    st = _lib().nvfp4_quantize(_ptr(x), rows, cols, ld, along, mode, block, int(rht), rht_seed, sr_seed, stream_id,
+                               ctypes.byref(ct), ws.ptr, _stream(stream))
+    _check(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_quantize_dual(x: torch.Tensor, mode: int = RNE, rht_seed: int = 0, sr_seed: int = 0, stream_row: int = 0,
+                        stream_col: int = 0, out_row: NVFP4Tensor | None = None, out_col: NVFP4Tensor | None = None,
+                        ws: Workspace | None = None, stream=None):
+    rows, cols, ld = _bf16_2d(x)
+    out_row = out_row or NVFP4Tensor.empty(rows, cols, BLOCK_1x16, x.device)
+    out_col = out_col or NVFP4Tensor.empty(cols, rows, BLOCK_1x16, x.device)
+    ws = ws or default_workspace()
+    a, b = out_row.c(), out_col.c()
+    st = _lib().nvfp4_quantize_dual(_ptr(x), rows, cols, ld, mode, rht_seed, sr_seed, stream_row, stream_col,
+                                    ctypes.byref(a), ctypes.byref(b), ws.ptr, _stream(stream))
+    _check(st, "nvfp4_quantize_dual")
+    return out_row, out_col
+
+
+def nvfp4_quantize_weight(w: torch.Tensor, transposed: bool = True, out: NVFP4Tensor | None = None,
+                          out_t: NVFP4Tensor | None = None, ws: Workspace | None = None, stream=None):
+    rows, cols, ld = _bf16_2d(w)
+    out = out or NVFP4Tensor.empty(rows, cols, BLOCK_16x16, w.device)
+    if transposed:
+        out_t = out_t or NVFP4Tensor.empty(cols, rows, BLOCK_16x16, w.device)
+    ws = ws or default_workspace()
+    a = out.c()
+    b = out_t.c() if transposed else None
+    st = _lib().nvfp4_quantize_weight(_ptr(w), rows, cols, ld, ctypes.byref(a), ctypes.byref(b) if b else None,
+                                      ws.ptr, _stream(stream))
+    _check(st, "nvfp4_quantize_weight")
+    return (out, out_t) if transposed else out
+
+
+def nvfp4_transpose_2d(w: NVFP4Tensor, out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    out = out or NVFP4Tensor.empty(w.k, w.rows, BLOCK_16x16, w.codes.device)
+    a, b = w.c(), out.c()
+    _check(_lib().nvfp4_transpose_2d(ctypes.byref(a), ctypes.byref(b), _stream(stream)), "nvfp4_transpose_2d")
+    return out
+
+
+def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+               ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D[M][N] = s_tA s_tB * A . B^T (both K-major quantized forms)."""
+    M, N = a.rows, b.rows
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
+    code = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("output must be bf16 or fp32")
+    ws = ws or default_workspace()
+    ca, cb = a.c(), b.c()
+    st = _lib().nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), out.stride(0), code, ws.ptr, _stream(stream))
+    _check(st, "nvfp4_gemm")
+    return out
+
+
+def nvfp4_gelu_fwd(h: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = torch.empty_like(h) if out is None else out
+    _check(_lib().nvfp4_gelu_fwd(_ptr(h), _ptr(out), h.numel(), _stream(stream)), "nvfp4_gelu_fwd")
+    return out
+
+
+def nvfp4_gelu_bwd(h: torch.Tensor, dg: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = torch.empty_like(h) if out is None else out
+    _check(_lib().nvfp4_gelu_bwd(_ptr(h), _ptr(dg), _ptr(out), h.numel(), _stream(stream)), "nvfp4_gelu_bwd")
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# linear layer
+# ---------------------------------------------------------------------------------------
+class LinearContext:
+    """Caller-owned buffers of one NVFP4 linear layer y = x w^T (T tokens, d in, n out)."""
+
+    def __init__(self, T: int, d: int, n: int, rht_seed: int = 0, device=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.T, self.d, self.n = T, d, n
+        self.xq = NVFP4Tensor.empty(T, d, BLOCK_1x16, device)
+        self.xq_rht = NVFP4Tensor.empty(d, T, BLOCK_1x16, device)
+        self.wq = NVFP4Tensor.empty(n, d, BLOCK_16x16, device)
+        self.wqt = NVFP4Tensor.empty(d, n, BLOCK_16x16, device)
+        self.dyq = NVFP4Tensor.empty(T, n, BLOCK_1x16, device)
+        self.dyq_rht = NVFP4Tensor.empty(n, T, BLOCK_1x16, device)
+        self.ws = Workspace(device)
+        self.ctx = CLinearCtx(T, d, n, rht_seed, self.xq.c(), self.xq_rht.c(), self.wq.c(), self.wqt.c(),
+                              self.dyq.c(), self.dyq_rht.c(), self.ws.buf.data_ptr(), 0, 0)
+
+    @property
+    def w_cached(self) -> bool:
+        return bool(self.ctx.w_cached)
+
+    @w_cached.setter
+    def w_cached(self, v: bool):
+        self.ctx.w_cached = 1 if v else 0
+
+
+def nvfp4_linear_fwd(ctx: LinearContext, x: torch.Tensor, w: torch.Tensor | None, y: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    if y is None:
+        y = torch.empty((ctx.T, ctx.n), dtype=torch.bfloat16, device=x.device)
+    st = _lib().nvfp4_linear_fwd(_ptr(x), _ptr(w), _ptr(y), ctypes.byref(ctx.ctx), _stream(stream))
+    _check(st, "nvfp4_linear_fwd")
+    return y
+
+
+def nvfp4_linear_bwd(ctx: LinearContext, dy: torch.Tensor, sr_seed: int, dx: torch.Tensor | None = None,
+                     dw: torch.Tensor | None = None, stream=None):
+    if dx is None:
+        dx = torch.empty((ctx.T, ctx.d), dtype=torch.bfloat16, device=dy.device)
+    if dw is None:
+        dw = torch.empty((ctx.n, ctx.d), dtype=torch.float32, device=dy.device)
+    st = _lib().nvfp4_linear_bwd(_ptr(dy), sr_seed, _ptr(dx), _ptr(dw), ctypes.byref(ctx.ctx), _stream(stream))
+    _check(st, "nvfp4_linear_bwd")
+    return dx, dw

@@ -1,0 +1,427 @@
+// api.cu -- the C ABI of libnvfp4 (declared in include/nvfp4.h): argument validation and
+// kernel launches.  No allocation, no host synchronisation (except nvfp4_poll), no printing.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "nvfp4.h"
+#include "nvfp4_device.cuh"
+#include "nvfp4_internal.h"
+
+using namespace nvfp4;
+
+namespace {
+
+std::atomic<uint64_t> g_budget_ns{2000000000ull};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sm_100 check, cached per device
+nvfp4_status check_device() {
+    static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_UNSUPPORTED;
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return cached[dev] == 1 ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED;
+}
+
+nvfp4_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return NVFP4_OK;
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+}
+
+int64_t nkt_of(int64_t k) { return ((k >> 4) + 3) >> 2; }
+
+bool has_scale_padding(int64_t rows, int64_t k) { return (rows & 127) != 0 || ((k >> 4) & 3) != 0; }
+
+nvfp4_status check_form_buffers(const nvfp4_tensor* t, bool need_tiles) {
+    if (!t || !t->codes || !t->scales || !t->tensor_scale) return NVFP4_ERR_NULL;
+    if (need_tiles && !t->tile_scales) return NVFP4_ERR_NULL;
+    if (!aligned16(t->codes) || !aligned16(t->scales)) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
+}
+
+nvfp4_status check_input(const void* x, int64_t rows, int64_t cols, int64_t ld) {
+    if (rows < 0 || cols < 0) return NVFP4_ERR_SHAPE;
+    if (cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (ld < cols) return NVFP4_ERR_SHAPE;
+    if (rows > 0 && cols > 0) {
+        if (!x) return NVFP4_ERR_NULL;
+        if (!aligned16(x) || (ld % 8) != 0) return NVFP4_ERR_ALIGN;
+    }
+    return NVFP4_OK;
+}
+
+__global__ void set_f32_kernel(float* p, float v) { *p = v; }
+
+Workspace* ws_of(void* ws) { return reinterpret_cast<Workspace*>(ws); }
+
+cudaError_t reset_amax(void* ws, cudaStream_t s) {
+    return cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + offsetof(Workspace, amax_a), 0, 2 * sizeof(uint32_t), s);
+}
+
+}  // namespace
+
+namespace nvfp4 {
+
+uint32_t rht_signs_host(uint64_t seed) {
+    uint32_t c0 = 0, c1 = 0, c2 = NVFP4_STREAM_RHT, c3 = 0;
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0, p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c0 & 0xFFFFu;
+}
+
+}  // namespace nvfp4
+
+extern "C" {
+
+size_t nvfp4_codes_bytes(int64_t rows, int64_t k) { return (rows > 0 && k > 0) ? (size_t)(rows * (k / 2)) : 0; }
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t k) {
+    if (rows <= 0 || k <= 0) return 0;
+    return (size_t)(((rows + 127) / 128) * 128 * nkt_of(k) * 4);
+}
+
+size_t nvfp4_tile_scales_bytes(int64_t rows, int64_t k) {
+    return (rows > 0 && k > 0) ? (size_t)((rows / 16) * (k / 16)) : 0;
+}
+
+size_t nvfp4_workspace_bytes(void) { return sizeof(Workspace); }
+
+nvfp4_status nvfp4_workspace_init(void* ws, nvfp4_stream_t stream) {
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(Workspace), stream));
+}
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along, nvfp4_round mode,
+                            nvfp4_block block, int rht, uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_id,
+                            nvfp4_tensor* out, void* ws, nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
+    if (along != 0 && along != 1) return NVFP4_ERR_ARG;
+    if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
+    if (block != NVFP4_BLOCK_1x16 && block != NVFP4_BLOCK_16x16) return NVFP4_ERR_ARG;
+    if (rht && (block == NVFP4_BLOCK_16x16 || along == 0)) return NVFP4_ERR_ARG;  // RHT: wgrad (along=1) forms only
+    const bool b16 = block == NVFP4_BLOCK_16x16;
+    if (nvfp4_status st = check_form_buffers(out, b16)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if ((along == 1 || b16) && (rows % 16) != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    const int64_t R = along ? cols : rows, K = along ? rows : cols;
+    out->rows = R;
+    out->k = K;
+    out->block = block;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (R == 0 || K == 0) {
+        set_f32_kernel<<<1, 1, 0, s>>>(out->tensor_scale, 1.0f);
+        return from_cuda(cudaGetLastError());
+    }
+    Workspace* w = ws_of(ws);
+    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+    if (has_scale_padding(R, K))
+        if (cudaError_t e = cudaMemsetAsync(out->scales, 0, nvfp4_scales_bytes(R, K), s)) return from_cuda(e);
+    const uint32_t signs = rht ? rht_signs_host(rht_seed) : 0u;
+    const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+    cudaError_t e = (along == 1 && rht) ? launch_amax_rht(xb, rows, cols, ldx, signs, &w->amax_a, &w->amax_b, &w->flags, s)
+                                        : launch_amax_plain(xb, rows, cols, ldx, &w->amax_a, &w->flags, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    QuantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = xb;
+    p.rows = rows;
+    p.cols = cols;
+    p.ld = ldx;
+    p.block16 = b16 ? 1 : 0;
+    p.signs = signs;
+    p.sr_seed = sr_seed;
+    if (along == 0) {
+        p.codes_row = out->codes;
+        p.scales_row = out->scales;
+        p.tiles_row = b16 ? out->tile_scales : nullptr;
+        p.st_row = out->tensor_scale;
+        p.amax_row = &w->amax_a;
+        p.nkt_row = nkt_of(K);
+        p.sr_row = mode == NVFP4_SR;
+        p.stream_row = stream_id;
+    } else {
+        p.codes_col = out->codes;
+        p.scales_col = out->scales;
+        p.tiles_col = b16 ? out->tile_scales : nullptr;
+        p.st_col = out->tensor_scale;
+        p.amax_col = rht ? &w->amax_b : &w->amax_a;
+        p.nkt_col = nkt_of(K);
+        p.sr_col = mode == NVFP4_SR;
+        p.rht_col = rht ? 1 : 0;
+        p.stream_col = stream_id;
+    }
+    return from_cuda(launch_quantize_tiles(p, s));
+}
+
+nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
+                                 uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
+                                 nvfp4_tensor* out_row, nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
+    if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
+    if (nvfp4_status st = check_form_buffers(out_row, false)) return st;
+    if (nvfp4_status st = check_form_buffers(out_col, false)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    out_row->rows = rows;
+    out_row->k = cols;
+    out_row->block = NVFP4_BLOCK_1x16;
+    out_col->rows = cols;
+    out_col->k = rows;
+    out_col->block = NVFP4_BLOCK_1x16;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0 || cols == 0) {
+        set_f32_kernel<<<1, 1, 0, s>>>(out_row->tensor_scale, 1.0f);
+        set_f32_kernel<<<1, 1, 0, s>>>(out_col->tensor_scale, 1.0f);
+        return from_cuda(cudaGetLastError());
+    }
+    Workspace* w = ws_of(ws);
+    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+    if (has_scale_padding(rows, cols))
+        if (cudaError_t e = cudaMemsetAsync(out_row->scales, 0, nvfp4_scales_bytes(rows, cols), s)) return from_cuda(e);
+    if (has_scale_padding(cols, rows))
+        if (cudaError_t e = cudaMemsetAsync(out_col->scales, 0, nvfp4_scales_bytes(cols, rows), s)) return from_cuda(e);
+    const uint32_t signs = rht_signs_host(rht_seed);
+    const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+    if (cudaError_t e = launch_amax_rht(xb, rows, cols, ldx, signs, &w->amax_a, &w->amax_b, &w->flags, s))
+        return from_cuda(e);
+    QuantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = xb;
+    p.rows = rows;
+    p.cols = cols;
+    p.ld = ldx;
+    p.signs = signs;
+    p.sr_seed = sr_seed;
+    p.codes_row = out_row->codes;
+    p.scales_row = out_row->scales;
+    p.st_row = out_row->tensor_scale;
+    p.amax_row = &w->amax_a;
+    p.nkt_row = nkt_of(cols);
+    p.sr_row = mode == NVFP4_SR;
+    p.stream_row = stream_row;
+    p.codes_col = out_col->codes;
+    p.scales_col = out_col->scales;
+    p.st_col = out_col->tensor_scale;
+    p.amax_col = &w->amax_b;
+    p.nkt_col = nkt_of(rows);
+    p.sr_col = mode == NVFP4_SR;
+    p.rht_col = 1;
+    p.stream_col = stream_col;
+    return from_cuda(launch_quantize_tiles(p, s));
+}
+
+nvfp4_status nvfp4_quantize_weight(const void* wp, int64_t rows, int64_t cols, int64_t ldw, nvfp4_tensor* w_q,
+                                   nvfp4_tensor* w_qt, void* ws, nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(wp, rows, cols, ldw)) return st;
+    if (nvfp4_status st = check_form_buffers(w_q, true)) return st;
+    if (w_qt)
+        if (nvfp4_status st = check_form_buffers(w_qt, false)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    w_q->rows = rows;
+    w_q->k = cols;
+    w_q->block = NVFP4_BLOCK_16x16;
+    if (w_qt) {
+        w_qt->rows = cols;
+        w_qt->k = rows;
+        w_qt->block = NVFP4_BLOCK_16x16;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (rows == 0 || cols == 0) {
+        set_f32_kernel<<<1, 1, 0, s>>>(w_q->tensor_scale, 1.0f);
+        if (w_qt) set_f32_kernel<<<1, 1, 0, s>>>(w_qt->tensor_scale, 1.0f);
+        return from_cuda(cudaGetLastError());
+    }
+    Workspace* w = ws_of(ws);
+    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+    if (has_scale_padding(rows, cols))
+        if (cudaError_t e = cudaMemsetAsync(w_q->scales, 0, nvfp4_scales_bytes(rows, cols), s)) return from_cuda(e);
+    if (w_qt && has_scale_padding(cols, rows))
+        if (cudaError_t e = cudaMemsetAsync(w_qt->scales, 0, nvfp4_scales_bytes(cols, rows), s)) return from_cuda(e);
+    const uint16_t* xb = reinterpret_cast<const uint16_t*>(wp);
+    if (cudaError_t e = launch_amax_plain(xb, rows, cols, ldw, &w->amax_a, &w->flags, s)) return from_cuda(e);
+    QuantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = xb;
+    p.rows = rows;
+    p.cols = cols;
+    p.ld = ldw;
+    p.block16 = 1;
+    p.codes_row = w_q->codes;
+    p.scales_row = w_q->scales;
+    p.tiles_row = w_q->tile_scales;
+    p.st_row = w_q->tensor_scale;
+    p.amax_row = &w->amax_a;
+    p.nkt_row = nkt_of(cols);
+    if (w_qt) {
+        p.codes_col = w_qt->codes;
+        p.scales_col = w_qt->scales;
+        p.tiles_col = w_qt->tile_scales;
+        p.st_col = w_qt->tensor_scale;
+        p.amax_col = &w->amax_a;
+        p.nkt_col = nkt_of(rows);
+    }
+    return from_cuda(launch_quantize_tiles(p, s));
+}
+
+nvfp4_status nvfp4_transpose_2d(const nvfp4_tensor* w, nvfp4_tensor* wt, nvfp4_stream_t stream) {
+    if (!w || !wt) return NVFP4_ERR_NULL;
+    if (nvfp4_status st = check_form_buffers(w, true)) return st;
+    if (nvfp4_status st = check_form_buffers(wt, false)) return st;
+    if (w->block != NVFP4_BLOCK_16x16) return NVFP4_ERR_ARG;
+    const int64_t R = w->rows, K = w->k;
+    if (R < 0 || K < 0 || R % 16 || K % 16) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    wt->rows = K;
+    wt->k = R;
+    wt->block = NVFP4_BLOCK_16x16;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (R == 0 || K == 0) {
+        set_f32_kernel<<<1, 1, 0, s>>>(wt->tensor_scale, 1.0f);
+        return from_cuda(cudaGetLastError());
+    }
+    if (has_scale_padding(K, R))
+        if (cudaError_t e = cudaMemsetAsync(wt->scales, 0, nvfp4_scales_bytes(K, R), s)) return from_cuda(e);
+    return from_cuda(launch_transpose_2d(w->codes, w->tile_scales, R, K, wt->codes, wt->scales, wt->tile_scales,
+                                         w->tensor_scale, wt->tensor_scale, s));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, int64_t ldd, nvfp4_dtype out_dtype,
+                        void* ws, nvfp4_stream_t stream) {
+    if (!a || !b || !d) return NVFP4_ERR_NULL;
+    if (nvfp4_status st = check_form_buffers(a, false)) return st;
+    if (nvfp4_status st = check_form_buffers(b, false)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32) return NVFP4_ERR_ARG;
+    const int64_t M = a->rows, N = b->rows, K = a->k;
+    if (b->k != K) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return NVFP4_ERR_LIMIT;
+    const int64_t esz = out_dtype == NVFP4_OUT_FP32 ? 4 : 2;
+    if (ldd < N) return NVFP4_ERR_SHAPE;
+    if (!aligned16(d) || (ldd * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gemm_nvf4(a->codes, a->scales, a->tensor_scale, M, b->codes, b->scales, b->tensor_scale, N, K,
+                                      d, ldd, out_dtype == NVFP4_OUT_FP32, &ws_of(ws)->flags, g_budget_ns.load(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static nvfp4_status check_ctx(const nvfp4_linear_ctx* c) {
+    if (!c) return NVFP4_ERR_NULL;
+    if (c->T <= 0 || c->d <= 0 || c->n <= 0) return NVFP4_ERR_SHAPE;
+    if (c->T % 64 || c->d % 64 || c->n % 64) return NVFP4_ERR_SHAPE;
+    if (!c->ws) return NVFP4_ERR_WORKSPACE;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linear_ctx* ctx, nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_ctx(ctx)) return st;
+    if (!x || !y || (!w && !ctx->w_cached)) return NVFP4_ERR_NULL;
+    nvfp4_status st;
+    if (!ctx->w_cached) {
+        st = nvfp4_quantize_weight(w, ctx->n, ctx->d, ctx->d, &ctx->wq, &ctx->wqt, ctx->ws, stream);
+        if (st) return st;
+    }
+    st = nvfp4_quantize_dual(x, ctx->T, ctx->d, ctx->d, NVFP4_RNE, ctx->rht_seed, 0, 0, 0, &ctx->xq, &ctx->xq_rht, ctx->ws,
+                             stream);
+    if (st) return st;
+    return nvfp4_gemm(&ctx->xq, &ctx->wq, y, ctx->n, NVFP4_OUT_BF16, ctx->ws, stream);
+}
+
+nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float* dw, nvfp4_linear_ctx* ctx,
+                              nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_ctx(ctx)) return st;
+    if (!dy) return NVFP4_ERR_NULL;
+    nvfp4_status st = nvfp4_quantize_dual(dy, ctx->T, ctx->n, ctx->n, NVFP4_SR, ctx->rht_seed, sr_seed, NVFP4_STREAM_DGRAD,
+                                          NVFP4_STREAM_WGRAD, &ctx->dyq, &ctx->dyq_rht, ctx->ws, stream);
+    if (st) return st;
+    if (dx) {
+        st = nvfp4_gemm(&ctx->dyq, &ctx->wqt, dx, ctx->d, NVFP4_OUT_BF16, ctx->ws, stream);
+        if (st) return st;
+    }
+    if (dw) {
+        st = nvfp4_gemm(&ctx->dyq_rht, &ctx->xq_rht, dw, ctx->d, NVFP4_OUT_FP32, ctx->ws, stream);
+        if (st) return st;
+    }
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gelu_fwd(const void* h, void* g, int64_t n, nvfp4_stream_t stream) {
+    if (n < 0) return NVFP4_ERR_SHAPE;
+    if (n == 0) return NVFP4_OK;
+    if (!h || !g) return NVFP4_ERR_NULL;
+    if (!aligned16(h) || !aligned16(g)) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gelu_fwd(reinterpret_cast<const uint16_t*>(h), reinterpret_cast<uint16_t*>(g), n,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n, nvfp4_stream_t stream) {
+    if (n < 0) return NVFP4_ERR_SHAPE;
+    if (n == 0) return NVFP4_OK;
+    if (!h || !dg || !dh) return NVFP4_ERR_NULL;
+    if (!aligned16(h) || !aligned16(dg) || !aligned16(dh)) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gelu_bwd(reinterpret_cast<const uint16_t*>(h), reinterpret_cast<const uint16_t*>(dg),
+                                     reinterpret_cast<uint16_t*>(dh), n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream) {
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+    uint32_t flags = 0;
+    if (cudaMemcpy(&flags, ws, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+    if (flags && cudaMemset(ws, 0, sizeof(uint32_t)) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+    if (flags & kFlagTimeout) return NVFP4_ERR_TIMEOUT;
+    if (flags & kFlagNonFinite) return NVFP4_ERR_NONFINITE;
+    return NVFP4_OK;
+}
+
+void nvfp4_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns ? ns : 2000000000ull); }
+
+const char* nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_NULL: return "a required pointer is NULL";
+        case NVFP4_ERR_ALIGN: return "a pointer or leading dimension is not 16-byte aligned";
+        case NVFP4_ERR_SHAPE: return "a size violates the call's shape rule";
+        case NVFP4_ERR_ARG: return "an argument is out of range or operands are inconsistent";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing";
+        case NVFP4_ERR_CUDA: return "a CUDA launch or runtime call failed";
+        case NVFP4_ERR_NONFINITE: return "NaN or Inf in a quantized input";
+        case NVFP4_ERR_TIMEOUT: return "a device-side wait ran out of its time budget";
+        case NVFP4_ERR_UNSUPPORTED: return "device is not sm_100 (B200)";
+        case NVFP4_ERR_LIMIT: return "a size exceeds a fixed limit of the call";
+    }
+    return "unknown status";
+}
+
+int nvfp4_version(void) { return 1; }
+
+}  // extern "C"

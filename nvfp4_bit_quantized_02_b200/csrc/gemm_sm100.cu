@@ -1,0 +1,416 @@
+// gemm_sm100.cu -- block-scaled NVFP4 GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// D[M][N] = s_tA * s_tB * sum_k (qA[m][k] * sA[m][k/16]) * (qB[n][k] * sB[n][k/16])
+// with E2M1 codes q, E4M3 block scales s and fp32 tensor scales s_t (gist.science "Pretraining
+// Large Language Models with NVFP4", 2.A; the FP4 GEMMs of the linear layers are the hot
+// spot, brainai.pro "Details techniques").
+//
+// One CTA computes a 128 x 256 output tile (one SM; 1 CTA per SM by shared memory):
+//   warp 0      TMA producer: per 256-wide K block, the A tile (128 rows x 128 bytes) and the
+//               B tile (256 x 128 bytes) by cp.async.bulk.tensor with 128-byte swizzle, and the
+//               matching 512-byte scale tiles by cp.async.bulk, into a 4-stage ring;
+//   warp 1      allocates 512 TMEM columns; one thread moves each stage's scales into TMEM
+//               (tcgen05.cp 32x128b.warpx4) and issues tcgen05.mma kind::mxf4nvf4
+//               block_scale scale_vec::4X (M=128, N=256, K=64), accumulating in fp32 in TMEM;
+//               tcgen05.commit frees the stage;
+//   warps 2-5   epilogue: tcgen05.ld 32x32b, times s_tA*s_tB, bf16 or fp32 stores.
+// TMEM columns: [0, 256) accumulator; per stage s, [256 + 48 s, +16) scales of A (4 columns per
+// 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).
+// Every mbarrier wait is bounded by a %globaltimer budget; on expiry the CTA raises the timeout
+// flag, drains its copies and MMAs (again bounded) and frees its TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "nvfp4_internal.h"
+
+namespace nvfp4 {
+
+constexpr int kBM = 128, kBN = 256, kBK = 256;  // K in elements (128 bytes of codes)
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK / 2;                 // 16384
+constexpr int kBBytes = kBN * kBK / 2;                 // 32768
+constexpr int kSFABytes = (kBM / 128) * (kBK / 64) * 512;  // 2048
+constexpr int kSFBBytes = (kBN / 128) * (kBK / 64) * 512;  // 4096
+constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // 55296 (54 KiB)
+constexpr int kBarrierBytes = 256;
+constexpr int kGemmSmem = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCol0 = 256, kSfColsPerStage = 48;
+
+static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment for the 128B swizzle");
+static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
+
+// instruction descriptor: dense, A/B = E2M1 (format 1 of the mxf4 kinds), both K-major,
+// N >> 3 at bit 17, scale type UE4M3 (bit 23 = 0), M >> 4 at bit 24, scale ids 0
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait.  Returns false if the CTA aborted (another role timed out) or this wait ran out
+// of its budget (then it raises the abort and the timeout flag).  `honor_abort` = false is used
+// by the drain after an abort, which must still see copies land.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint32_t* flags, uint64_t budget_ns, bool honor_abort = true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (honor_abort && *abort) return false;
+        if (globaltimer() - t0 > budget_ns) {
+            *abort = 1u;
+            atomicOr(flags, kFlagTimeout);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups 1024 bytes apart
+// (stride byte offset), leading byte offset unused (1), descriptor version 1 (bit 46),
+// layout type 2 = SWIZZLE_128B (bits 61-63)
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+// descriptor of one 512-byte scale tile for tcgen05.cp 32x128b: 32 rows of 16 bytes, no swizzle,
+// core matrices (8 rows x 16 bytes) contiguous: both byte offsets 128
+__device__ __forceinline__ uint64_t desc_sf_tile(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+           (1ull << 46);
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------------------
+struct GemmParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* sta;
+    const float* stb;
+    void* d;
+    int64_t ldd;
+    int32_t out_fp32;
+    int32_t M, N, K;
+    int32_t nkt;        // ceil(K / 64): 64-wide K steps (= scale tiles per 128-row tile)
+    int32_t num_kb;     // ceil(K / 256): pipeline stages' worth of K
+    int32_t sfb_row_tiles;  // ceil(N / 128)
+    uint32_t* flags;
+    uint64_t budget_ns;
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* bar_area = smem + kStages * kStageBytes;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
+    uint64_t* empty_bar = full_bar + kStages;
+    uint64_t* accum_bar = empty_bar + kStages;
+    uint64_t* done_bar = accum_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+
+    // zero the scale regions once: a B tile past the last 128-row scale tile is never loaded
+    // and must read as zero scales (its codes are zero-filled by TMA)
+    for (int i = threadIdx.x; i < kStages * (kSFABytes + kSFBBytes) / 16; i += kGemmThreads) {
+        const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
+        reinterpret_cast<uint4*>(smem + s * kStageBytes + kABytes + kBBytes)[o] = make_uint4(0, 0, 0, 0);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        mbar_init(smem_u32(accum_bar), 1);
+        mbar_init(smem_u32(done_bar), 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------- producer -------------------------------------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            const int rt_a = m0 >> 7;
+            int issued = 0;
+            for (int kb = 0; kb < p.num_kb; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+                if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
+                const int steps = min(4, p.nkt - 4 * kb);
+                const uint32_t sf_bytes = (uint32_t)steps * 512u;
+                int btiles = 0;
+                for (int t = 0; t < 2; ++t) btiles += ((n0 >> 7) + t < p.sfb_row_tiles) ? 1 : 0;
+                const uint32_t full = smem_u32(&full_bar[s]);
+                mbar_expect_tx(full, (uint32_t)(kABytes + kBBytes) + sf_bytes * (uint32_t)(1 + btiles));
+                uint8_t* st = smem + s * kStageBytes;
+                tma_load_2d(smem_u32(st), &tmA, kb * 128, m0, full);
+                tma_load_2d(smem_u32(st + kABytes), &tmB, kb * 128, n0, full);
+                bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + ((int64_t)rt_a * p.nkt + 4 * kb) * 512, sf_bytes, full);
+                for (int t = 0; t < 2; ++t) {
+                    const int rt = (n0 >> 7) + t;
+                    if (rt < p.sfb_row_tiles)
+                        bulk_load(smem_u32(st + kABytes + kBBytes + kSFABytes + t * 2048),
+                                  p.sfb + ((int64_t)rt * p.nkt + 4 * kb) * 512, sf_bytes, full);
+                }
+                ++issued;
+            }
+            if (*abort_flag) {
+                // drain: every copy this thread issued must land before the CTA exits
+                for (int kb = max(0, issued - kStages); kb < issued; ++kb)
+                    mbar_wait(smem_u32(&full_bar[kb % kStages]), (uint32_t)(kb / kStages) & 1u, abort_flag, p.flags,
+                              p.budget_ns, false);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer -----------------------------------------
+        if (lane == 0) {
+            const uint32_t sbase = smem_u32(smem);
+            int kb = 0;
+            for (; kb < p.num_kb; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+                if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) break;
+                tc_fence_after();
+                const int steps = min(4, p.nkt - 4 * kb);
+                const uint32_t a_s = sbase + s * kStageBytes;
+                const uint32_t b_s = a_s + kABytes;
+                const uint32_t sfa_s = b_s + kBBytes;
+                const uint32_t sfb_s = sfa_s + kSFABytes;
+                const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
+                const uint32_t t_sfb = t_sfa + 16;
+                for (int j = 0; j < steps; ++j) {
+                    tmem_cp_sf(t_sfa + 4 * j, desc_sf_tile(sfa_s + 512 * j));
+                    tmem_cp_sf(t_sfb + 8 * j, desc_sf_tile(sfb_s + 512 * j));
+                    tmem_cp_sf(t_sfb + 8 * j + 4, desc_sf_tile(sfb_s + 2048 + 512 * j));
+                }
+                for (int j = 0; j < steps; ++j) {
+                    mma_nvf4(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), kIdesc, t_sfa + 4 * j,
+                             t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&empty_bar[s]));
+            }
+            if (kb == p.num_kb) mma_commit(smem_u32(accum_bar));
+            // all MMAs of this thread complete before TMEM may be freed
+            mma_commit(smem_u32(done_bar));
+            mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+        }
+    } else {
+        // ------------------------------- epilogue (warps 2..5) ------------------------------
+        const int q = warp & 3;  // TMEM lane quadrant this warp may read
+        const int row = m0 + q * 32 + lane;
+        const bool ok = mbar_wait(smem_u32(accum_bar), 0u, abort_flag, p.flags, p.budget_ns);
+        __syncwarp();
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            tc_fence_after();
+            const float alpha = __fmul_rn(*p.sta, *p.stb);
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
+                tmem_ld_wait();
+                const int col0 = n0 + c * 32;
+                if (row < p.M && col0 < p.N) {
+                    const bool full_chunk = col0 + 32 <= p.N;
+                    if (p.out_fp32) {
+                        float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
+                        if (full_chunk) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                reinterpret_cast<float4*>(out)[j] = make_float4(
+                                    __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
+                                    __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+                        }
+                    } else {
+                        uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
+                        uint32_t w[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
+                            float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                            uint32_t v;
+                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
+                            w[j] = v;
+                        }
+                        if (full_chunk) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 2D map over codes [rows][k/2] bytes, box = 128 bytes x box_rows, 128-byte swizzle, zero fill
+static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
+                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
+                             void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
+                             cudaStream_t stream) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap ta, tb;
+    if (!make_code_map(&ta, a_codes, M, K, kBM) || !make_code_map(&tb, b_codes, N, K, kBN))
+        return cudaErrorInvalidValue;
+    GemmParams p;
+    p.sfa = a_scales;
+    p.sfb = b_scales;
+    p.sta = a_st;
+    p.stb = b_st;
+    p.d = d;
+    p.ldd = ldd;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.M = (int32_t)M;
+    p.N = (int32_t)N;
+    p.K = (int32_t)K;
+    p.nkt = (int32_t)((K + 63) / 64);
+    p.num_kb = (int32_t)((K + kBK - 1) / kBK);
+    p.sfb_row_tiles = (int32_t)((N + 127) / 128);
+    p.flags = flags;
+    p.budget_ns = budget_ns;
+    dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM));
+    gemm_nvf4_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4

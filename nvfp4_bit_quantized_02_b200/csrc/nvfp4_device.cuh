@@ -1,0 +1,175 @@
+// nvfp4_device.cuh -- device primitives of the NVFP4 quantization path (sm_100a).
+//
+// Number formats (gist.science "Pretraining Large Language Models with NVFP4", Technische
+// Zusammenfassung 2.A): E2M1 elements, E4M3 block scales, an fp32 tensor scale.  Rounding
+// (2.B.4): round-to-nearest-even, or stochastic rounding for gradients.  Rotation (2.B.2): a
+// seeded 16-point Random Hadamard Transform.
+//
+// Every fp32 operation whose result decides a code is written as one IEEE operation in
+// round-to-nearest (explicit __fdiv_rn / __fmul_rn / __fadd_rn / __fsub_rn), so that codes
+// and scales are reproducible bit for bit.
+#pragma once
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+// ---------------------------------------------------------------------------------------
+// bf16 unpacking (bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 bits)
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t pair) { return __uint_as_float(pair << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t pair) { return __uint_as_float(pair & 0xFFFF0000u); }
+
+// fp32 -> bf16 bits, round to nearest even (hardware cvt).
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// E2M1 encode, round-to-nearest-even, saturating to +-6, sign kept.  Two values per
+// instruction; `lo` lands in bits [0,4), `hi` in bits [4,8).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// E2M1 stochastic rounding.  For |u| in [lo, hi) of the grid {0,.5,1,1.5,2,3,4,6} the value
+// goes up iff r16 < ceil(((|u| - lo) / (hi - lo)) * 2^16); |u| >= 6 gives 6; sign kept.
+// The fraction is read straight from the fp32 bits (all quantities are exact):
+//   |u| in [1, 6):   lo keeps the exponent and the top mantissa bit, step = 2^(e-1), so
+//                    f * 2^16 = (mantissa & 0x3FFFFF) / 2^6;
+//   |u| in [.5, 1):  lo = .5, step = .5, f * 2^16 = mantissa / 2^7;
+//   |u| in [0, .5):  lo = 0, step = .5, f * 2^16 = |u| * 2^17 (exact power-of-two scaling).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */) {
+    if (a >= 0x3F800000u) return ((a & 0x3FFFFFu) + 63u) >> 6;
+    if (a >= 0x3F000000u) return ((a & 0x7FFFFFu) + 127u) >> 7;
+    return (uint32_t)ceilf(__fmul_rn(__uint_as_float(a), 131072.0f));
+}
+
+__device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
+    const uint32_t b = __float_as_uint(u);
+    const uint32_t sign = (b >> 28) & 8u;
+    const uint32_t a = b & 0x7FFFFFFFu;
+    if (a >= 0x40C00000u) return sign | 7u;   // |u| >= 6 (and +-inf)
+    uint32_t code;
+    if (a >= 0x3F800000u) code = 2u + 2u * ((a >> 23) - 127u) + ((a >> 22) & 1u);
+    else code = (a >= 0x3F000000u) ? 1u : 0u;
+    return sign | (code + (r16 < e2m1_sr_threshold(a) ? 1u : 0u));
+}
+
+// ---------------------------------------------------------------------------------------
+// E4M3 ("fn": no infinities, 0x7F = NaN) for non-negative block scales
+// ---------------------------------------------------------------------------------------
+// Round-to-nearest-even with saturation to 448 (hardware cvt, .satfinite).
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float y) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u16 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(0.0f), "f"(y));
+    return r & 0xFFu;
+}
+
+// Value of a non-negative, non-NaN code: m * 2^-9 for exponent field 0, else
+// (1 + m/8) * 2^(e-7), assembled directly as fp32 bits.
+__device__ __forceinline__ float e4m3_decode(uint32_t c) {
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : __fmul_rn((float)m, 0.001953125f);
+}
+
+// ---------------------------------------------------------------------------------------
+// Tensor-level scales (two-level scaling, 2.A): S_enc = 6*448/amax_t, s_t = amax_t/(6*448),
+// one IEEE division each; an all-zero tensor gets 1 and 1.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float encode_scale(float amax_t) {
+    return amax_t > 0.0f ? __fdiv_rn(2688.0f, amax_t) : 1.0f;
+}
+__device__ __forceinline__ float decode_scale(float amax_t) {
+    return amax_t > 0.0f ? __fdiv_rn(amax_t, 2688.0f) : 1.0f;
+}
+
+// Block scale from the block amax: E4M3(RNE, sat)( (amax_b / 6) * S_enc ), and the element
+// multiplier r_b = S_enc / dec(s_b) (0 for a zero scale).
+struct BlockScale {
+    uint32_t code;
+    float mult;
+};
+__device__ __forceinline__ BlockScale block_scale(float amax_b, float s_enc) {
+    BlockScale s;
+    s.code = e4m3_rne_sat(__fmul_rn(__fdiv_rn(amax_b, 6.0f), s_enc));
+    s.mult = s.code ? __fdiv_rn(s_enc, e4m3_decode(s.code)) : 0.0f;
+    return s;
+}
+
+// ---------------------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11).  Counter (c0, c1, c2, c3), key (k0, k1).
+// ---------------------------------------------------------------------------------------
+struct U4 {
+    uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                            uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return U4{c0, c1, c2, c3};
+}
+
+// The four 32-bit words for element group g = i/8 of stream `stream_id`.
+__device__ __forceinline__ U4 sr_words(uint64_t seed, uint32_t stream_id, uint64_t g) {
+    return philox4x32_10((uint32_t)g, (uint32_t)(g >> 32), stream_id, 0u, (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+}
+
+// ---------------------------------------------------------------------------------------
+// 16-point Random Hadamard Transform: v <- 0.25 * H16 * (D v), D = diag(signs), the butterfly
+// stages h = 1, 2, 4, 8 in that order, each pair (i, i+h) with bit h of i clear becoming
+// (a + b, a - b).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void rht16(float (&v)[16], uint32_t signs) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = ((signs >> j) & 1u) ? -v[j] : v[j];
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            const float a = v[i], b = v[i + h];
+            v[i] = __fadd_rn(a, b);
+            v[i + h] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+}
+
+// ---------------------------------------------------------------------------------------
+// Position of the scale of (form row r, K-block kb) in the 128x4-tile layout read by the
+// tcgen05 block-scaled MMA.
+// ---------------------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, int64_t nkt) {
+    return ((r >> 7) * nkt + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,68 @@
+// nvfp4_internal.h -- declarations shared by the CUDA translation units of libnvfp4.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+// workspace layout (256 bytes, caller-owned device memory)
+struct Workspace {
+    uint32_t flags;       // kFlag* bits, sticky until nvfp4_poll
+    uint32_t amax_a;      // fp32 bits: plain amax of the last quantize call
+    uint32_t amax_b;      // fp32 bits: amax after the RHT
+    uint32_t pad[61];
+};
+static_assert(sizeof(Workspace) == 256, "workspace is 256 bytes");
+
+constexpr uint32_t kFlagNonFinite = 1u;
+constexpr uint32_t kFlagTimeout = 2u;
+
+// parameters of the tile quantizer (one read of x, up to two forms)
+struct QuantParams {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    int32_t block16;  // 1: 16x16 tiles (both forms share the tile scale)
+    // ROW form: K = cols
+    uint8_t* codes_row;
+    uint8_t* scales_row;
+    uint8_t* tiles_row;
+    float* st_row;
+    const uint32_t* amax_row;
+    int64_t nkt_row;
+    int32_t sr_row;
+    uint32_t stream_row;
+    // COL form: K = rows (the transposed operand)
+    uint8_t* codes_col;
+    uint8_t* scales_col;
+    uint8_t* tiles_col;
+    float* st_col;
+    const uint32_t* amax_col;
+    int64_t nkt_col;
+    int32_t sr_col;
+    int32_t rht_col;
+    uint32_t stream_col;
+    uint32_t signs;
+    uint64_t sr_seed;
+};
+
+cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax,
+                              uint32_t* flags, cudaStream_t s);
+cudaError_t launch_amax_rht(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t signs,
+                            uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags, cudaStream_t s);
+cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s);
+cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* tiles, int64_t R, int64_t K, uint8_t* codes_t,
+                                uint8_t* scales_t, uint8_t* tiles_t, const float* st_in, float* st_out,
+                                cudaStream_t s);
+cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
+                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
+                             void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
+                             cudaStream_t stream);
+cudaError_t launch_gelu_fwd(const uint16_t* h, uint16_t* g, int64_t n, cudaStream_t s);
+cudaError_t launch_gelu_bwd(const uint16_t* h, const uint16_t* dg, uint16_t* dh, int64_t n, cudaStream_t s);
+
+// host-side Philox4x32-10 (same algorithm as the device one) for the RHT sign draw
+uint32_t rht_signs_host(uint64_t seed);
+
+}  // namespace nvfp4

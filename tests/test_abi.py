@@ -1,0 +1,93 @@
+"""The C-ABI library loads on a machine without a GPU and exports every entry point that
+include/nvfp4.h declares; host-only calls (sizes, status strings) and argument validation
+work without touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import nvfp4_bit_quantized_02_b200 as nv
+    if not os.path.exists(nv.LIB_PATH):
+        from nvfp4_bit_quantized_02_b200.csrc import build as b
+        b.build()
+    return nv.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 15
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_sizes(L):
+    assert L.nvfp4_codes_bytes(8192, 5120) == 8192 * 2560
+    assert L.nvfp4_scales_bytes(8192, 5120) == 8192 * 320
+    assert L.nvfp4_scales_bytes(200, 48) == 256 * 4       # rows to 128, K/16 to a multiple of 4
+    assert L.nvfp4_tile_scales_bytes(20480, 5120) == 1280 * 320
+    assert L.nvfp4_workspace_bytes() == 256
+    assert L.nvfp4_codes_bytes(0, 64) == 0
+
+
+def test_status_strings(L):
+    for s in range(11):
+        assert L.nvfp4_status_string(s)
+    assert L.nvfp4_status_string(0) == b"ok"
+    assert L.nvfp4_version() >= 1
+
+
+def test_validation_before_any_device_work(L):
+    import nvfp4_bit_quantized_02_b200 as nv
+    t = nv.CTensor(16, 16, 0, 16, 0, 0, 0, 0)
+    ws = ctypes.c_void_p(16)
+    x = ctypes.c_void_p(16)
+    # cols not a multiple of 16
+    assert L.nvfp4_quantize(x, 32, 24, 24, 0, 0, 0, 0, 0, 0, 0, ctypes.byref(t), ws, None) == 3
+    # misaligned input
+    assert L.nvfp4_quantize(ctypes.c_void_p(18), 32, 32, 32, 0, 0, 0, 0, 0, 0, 0, ctypes.byref(t), ws, None) == 2
+    # bad enums / RHT on a non-wgrad form
+    assert L.nvfp4_quantize(x, 32, 32, 32, 2, 0, 0, 0, 0, 0, 0, ctypes.byref(t), ws, None) == 4
+    assert L.nvfp4_quantize(x, 32, 32, 32, 0, 0, 0, 1, 0, 0, 0, ctypes.byref(t), ws, None) == 4
+    # 16x16 without tile scales
+    assert L.nvfp4_quantize(x, 32, 32, 32, 0, 0, 1, 0, 0, 0, 0, ctypes.byref(t), ws, None) == 1
+    # missing workspace
+    assert L.nvfp4_quantize(x, 32, 32, 32, 0, 0, 0, 0, 0, 0, 0, ctypes.byref(t), None, None) == 5
+    # along=1 needs rows % 16
+    assert L.nvfp4_quantize(x, 24, 32, 32, 1, 0, 0, 0, 0, 0, 0, ctypes.byref(t), ws, None) == 3
+    # GEMM: K mismatch, K % 32, null output, misaligned ldd
+    a = nv.CTensor(16, 16, 0, 16, 128, 64, 0, 0)
+    b = nv.CTensor(16, 16, 0, 16, 128, 96, 0, 0)
+    d = ctypes.c_void_p(16)
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, None) == 4
+    b.k = 48
+    a.k = 48
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, None) == 3
+    a.k = b.k = 64
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), None, 128, 0, ws, None) == 1
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 129, 0, ws, None) == 2
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 100, 0, ws, None) == 3
+    # linear: shapes must be multiples of 64
+    ctx = nv.CLinearCtx()
+    ctx.T, ctx.d, ctx.n, ctx.ws = 100, 64, 64, 16
+    assert L.nvfp4_linear_fwd(x, x, x, ctypes.byref(ctx), None) == 3
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import nvfp4_bit_quantized_02_b200 as nv
+    monkeypatch.setattr(nv, "_L", None)
+    monkeypatch.setattr(nv, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        nv.lib()

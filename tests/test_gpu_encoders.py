@@ -1,0 +1,108 @@
+"""The device encoders of the CUDA path against the CPU oracle, exhaustively over their input
+ranges, and the device Philox4x32-10 against the oracle and against cuRAND's independent
+Philox4_32_10 (which pins the oracle's generator to a third implementation)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import checks, parallel_map
+
+pytestmark = pytest.mark.gpu
+
+CHUNK = 1 << 26
+
+
+def _oracle_chunked(fn, x: np.ndarray, out_dtype):
+    out = np.empty(x.shape, out_dtype)
+    step = 1 << 21
+    def work(i):
+        out[i:i + step] = fn(x[i:i + step])
+    parallel_map(work, range(0, x.size, step))
+    return out
+
+
+def _sweep(lo_bits: int, hi_bits: int, gpu_fn, ora_fn, out_dtype, torch_dtype, transform=None):
+    for start in range(lo_bits, hi_bits, CHUNK):
+        n = min(CHUNK, hi_bits - start)
+        dev = torch.empty(n, dtype=torch_dtype, device="cuda")
+        assert gpu_fn(start, n, ctypes.c_void_p(dev.data_ptr())) == 0
+        got = dev.cpu().numpy()
+        x = (np.arange(n, dtype=np.uint64) + np.uint64(start)).astype(np.uint32).view(np.float32)
+        want = _oracle_chunked(ora_fn, x, out_dtype)
+        if transform is not None:
+            got = transform(got)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, f"bits {start + int(bad[0]):#010x}: gpu {got[bad[0]]} oracle {want[bad[0]]}"
+
+
+def test_e2m1_rne_all_finite_fp32():
+    L = checks()
+    both = lambda b: np.where((b & 15) == (b >> 4), b & 15, 255).astype(np.uint8)   # both nibbles must agree
+    for lo, hi in ((0x00000000, 0x7F800000), (0x80000000, 0xFF800000)):
+        _sweep(lo, hi, L.chk_e2m1_rne, oracle.e2m1_rne, np.uint8, torch.uint8, transform=both)
+
+
+def test_e2m1_sr_threshold_all_below_six():
+    L = checks()
+    _sweep(0x00000000, 0x40C00000, L.chk_e2m1_sr_threshold, oracle.e2m1_sr_threshold, np.uint32, torch.int32,
+           transform=lambda a: a.view(np.uint32))
+
+
+def test_e2m1_sr_codes_random():
+    L = checks()
+    rng = np.random.default_rng(3)
+    n = 1 << 22
+    x = (rng.standard_normal(n) * rng.choice([0.1, 1, 3, 10], n)).astype(np.float32)
+    r = rng.integers(0, 1 << 16, n, dtype=np.uint32)
+    xd, rd = torch.from_numpy(x).cuda(), torch.from_numpy(r.view(np.int32)).cuda()
+    out = torch.empty(n, dtype=torch.uint8, device="cuda")
+    assert L.chk_e2m1_sr(ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(rd.data_ptr()), n, ctypes.c_void_p(out.data_ptr())) == 0
+    assert np.array_equal(out.cpu().numpy(), oracle.e2m1_sr(x, r))
+
+
+def test_e4m3_all_nonnegative_fp32():
+    L = checks()
+    _sweep(0x00000000, 0x7F800001, L.chk_e4m3, oracle.e4m3_rne_sat, np.uint8, torch.uint8)
+
+
+def test_e4m3_decode_all_codes():
+    L = checks()
+    out = torch.empty(128, dtype=torch.float32, device="cuda")
+    assert L.chk_e4m3_decode(ctypes.c_void_p(out.data_ptr())) == 0
+    got = out.cpu().numpy()[:127].astype(np.float64)
+    want = np.array([oracle.e4m3_value(c) for c in range(127)])
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("seed,stream", [(0, 1), (0x123456789ABCDEF, 2), (2 ** 64 - 1, 3), (42, 0)])
+def test_philox_matches_oracle_and_curand(seed, stream):
+    L = checks()
+    n = 1 << 16
+    for g0 in (0, (1 << 32) - 5, 123456789012):
+        dev = torch.empty(4 * n, dtype=torch.int32, device="cuda")
+        cur = torch.empty(4 * n, dtype=torch.int32, device="cuda")
+        assert L.chk_philox(seed, stream, g0, n, ctypes.c_void_p(dev.data_ptr())) == 0
+        assert L.chk_curand_philox(seed, stream, g0, n, ctypes.c_void_p(cur.data_ptr())) == 0
+        ours = dev.cpu().numpy().view(np.uint32).reshape(n, 4)
+        theirs = cur.cpu().numpy().view(np.uint32).reshape(n, 4)
+        want = oracle.philox_blocks(seed, stream, g0, n)
+        assert np.array_equal(theirs, want), "oracle Philox disagrees with cuRAND"
+        assert np.array_equal(ours, want), "device Philox disagrees with the oracle"
+
+
+def test_rht16_matches_oracle_bit_exact():
+    L = checks()
+    rng = np.random.default_rng(8)
+    n = 4096
+    x = (rng.standard_normal((n, 16)) * rng.choice([1e-30, 1e-3, 1, 1e4], (n, 1))).astype(np.float32)
+    for seed in (0, 7, 99):
+        signs = oracle.rht_signs(seed)
+        xd = torch.from_numpy(x).cuda()
+        out = torch.empty_like(xd)
+        assert L.chk_rht16(ctypes.c_void_p(xd.data_ptr()), n, signs, ctypes.c_void_p(out.data_ptr())) == 0
+        got = out.cpu().numpy()
+        want = np.stack([oracle.rht16(r, signs) for r in x])
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
