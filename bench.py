@@ -1,0 +1,373 @@
+"""Benchmark of the NVFP4 linear layer (fprop + dgrad + wgrad with every quantize, RHT and
+transpose kernel) at T=8192 tokens, d=5120 in-features, n=20480 out-features on B200s.
+
+One step = nvfp4_linear_fwd (16x16 weight quantization + both activation forms + fprop GEMM)
+followed by nvfp4_linear_bwd (both SR gradient forms + dgrad GEMM + wgrad GEMM), on synthetic
+inputs resident in HBM.  value = 3 * 2 * T * d * n / step time (TFLOPS), whole job.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+N > 1 runs under torch.distributed.run (one rank per GPU, NCCL); each rank runs the full layer
+on its own batch (weak scaling).  --impl reference times the CPU oracle on this host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "NVFP4 linear fwd+bwd TFLOPS at 8192x5120x20480; quantize HBM GB/s"
+T_TOK, D_IN, D_OUT = 8192, 5120, 20480
+FLOP_STEP = 3 * 2 * T_TOK * D_IN * D_OUT
+FLOP_GEMM = 2 * T_TOK * D_IN * D_OUT
+# algorithmic bytes of one two-pass dual quantize call per input element:
+# 2 B read (amax) + 2 B read (quantize) + 2 forms x (0.5 B codes + 1/16 B scales)
+Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path:
+                try:
+                    os.remove(self.path)
+                except OSError:
+                    pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [int(r[1]) for r in rows]
+        smax = max(int(r[2]) for r in rows)
+        loaded = [r for r in rows if float(r[3] or 0) > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(int(r[1]) for r in loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded), "sm_mhz_min": min(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------------------
+def make_inputs(device):
+    import synth
+    x = synth.activations(T_TOK, D_IN, seed=0, outlier_frac=0.001)
+    w = synth.weights(D_OUT, D_IN, seed=1)
+    dy = synth.grad_output(T_TOK, D_OUT, seed=2)
+    return x, w, dy
+
+
+def run_ours(args, rank, world, local_rank):
+    import nvfp4_bit_quantized_02_b200 as nv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = torch.distributed if world > 1 else None
+    x_h, w_h, dy_h = make_inputs(dev)
+    x, w, dy = x_h.to(dev), w_h.to(dev), dy_h.to(dev)
+    ctx = nv.LinearContext(T_TOK, D_IN, D_OUT, rht_seed=0, device=dev)
+    y = torch.empty((T_TOK, D_OUT), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((T_TOK, D_IN), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    # Per-call events: the step is the sequence of the library's public calls that
+    # nvfp4_linear_fwd / nvfp4_linear_bwd make, timed one by one on the current stream.
+    def step(sr_seed, ev=None):
+        def rec(i):
+            if ev is not None:
+                ev[i].record()
+        rec(0)
+        nv.nvfp4_quantize_weight(w, out=ctx.wq, out_t=ctx.wqt, ws=ctx.ws)
+        rec(1)
+        nv.nvfp4_quantize_dual(x, mode=nv.RNE, rht_seed=0, out_row=ctx.xq, out_col=ctx.xq_rht, ws=ctx.ws)
+        rec(2)
+        nv.nvfp4_gemm(ctx.xq, ctx.wq, out=y, ws=ctx.ws)
+        rec(3)
+        nv.nvfp4_quantize_dual(dy, mode=nv.SR, rht_seed=0, sr_seed=sr_seed, stream_row=nv.STREAM_DGRAD,
+                               stream_col=nv.STREAM_WGRAD, out_row=ctx.dyq, out_col=ctx.dyq_rht, ws=ctx.ws)
+        rec(4)
+        nv.nvfp4_gemm(ctx.dyq, ctx.wqt, out=dx, ws=ctx.ws)
+        rec(5)
+        nv.nvfp4_gemm(ctx.dyq_rht, ctx.xq_rht, out=dw, ws=ctx.ws)
+        rec(6)
+
+    launches_per_step = 2 + 2 + 1 + 2 + 1 + 1   # amax+tile (W), amax+tile (X), fprop, amax+tile (dY), dgrad, wgrad
+
+    for i in range(args.warmup):
+        step(1000 + i)
+    torch.cuda.synchronize()
+    status = nv.nvfp4_poll(ctx.ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)                  # evict L2 between steps (outside the events)
+            step(k, events[k])
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    status = nv.nvfp4_poll(ctx.ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} during timing")
+
+    seg = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(6)] for k in range(args.steps)]
+    step_ms = [sum(s) for s in seg]
+    ms_total = sum(step_ms)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total_max = t.item()
+    ms_per_step = ms_total_max / args.steps
+
+    gemm_ms = [s[i] for s in seg for i in (2, 4, 5)]
+    q_ms = sum(s[0] + s[1] + s[3] for s in seg)
+    q_bytes = args.steps * Q_BYTES_PER_ELEM * (D_OUT * D_IN + T_TOK * D_IN + T_TOK * D_OUT)
+    peaks, peak_kind = load_peaks()
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    achieved = FLOP_GEMM / (gemm_avg_ms * 1e-3) / 1e12
+    peak_tensor = FP4_OVER_BF16 * peaks["bf16_tflops_sustained"]
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API from pinned host buffers ---------------------
+    e2e = None
+    if args.e2e_steps > 0:
+        hx, hw, hdy = (t.pin_memory() for t in (x_h, w_h, dy_h))
+        hy = torch.empty((T_TOK, D_OUT), dtype=torch.bfloat16).pin_memory()
+        hdx = torch.empty((T_TOK, D_IN), dtype=torch.bfloat16).pin_memory()
+        hdw = torch.empty((D_OUT, D_IN), dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
+        d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
+
+        def e2e_step(seed):
+            x.copy_(hx, non_blocking=True)
+            w.copy_(hw, non_blocking=True)
+            dy.copy_(hdy, non_blocking=True)
+            nv.nvfp4_linear_fwd(ctx, x, w, y)
+            nv.nvfp4_linear_bwd(ctx, dy, seed, dx, dw)
+            hy.copy_(y, non_blocking=True)
+            hdx.copy_(dx, non_blocking=True)
+            hdw.copy_(dw, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in range(args.e2e_steps):
+            e2e_step(k)
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if dist:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = te.item() / args.e2e_steps
+        e2e = {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW"}
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC,
+        "value": world * FLOP_STEP / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W, N(0,1e-4) dY; bf16)",
+        "config": {"workload": "NVFP4 linear fwd+bwd: fprop 8192x20480x5120, dgrad 8192x5120x20480, "
+                               "wgrad 20480x5120x8192, W 16x16 quantized every step",
+                   "tokens": T_TOK, "d_in": D_IN, "d_out": D_OUT, "rht": "16-point, wgrad operands",
+                   "sr": "Philox4x32-10, dY both forms",
+                   "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_kernel", "achieved": achieved,
+                     "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
+                     "traffic": None,
+                     "peak_basis": f"{FP4_OVER_BF16:g} x {peak_kind} sustained bf16 ({peaks['bf16_tflops_sustained']} TF/s)",
+                     "per_launch_flop": FLOP_GEMM, "avg_launch_ms": gemm_avg_ms},
+        "quantize": {"gbs": q_gbs, "unit": "GB/s", "peak_hbm_gbs": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
+                     "bytes_per_elem": Q_BYTES_PER_ELEM, "peak_basis": peak_kind,
+                     "per_call_ms": {"W": statistics.mean(s[0] for s in seg), "X": statistics.mean(s[1] for s in seg),
+                                     "dY": statistics.mean(s[3] for s in seg)}},
+        "gemm_tflops": {"fprop": FLOP_GEMM / statistics.mean(s[2] for s in seg) / 1e9,
+                        "dgrad": FLOP_GEMM / statistics.mean(s[4] for s in seg) / 1e9,
+                        "wgrad": FLOP_GEMM / statistics.mean(s[5] for s in seg) / 1e9},
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "impl": "ours",
+    }
+    if args.cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args)
+    return line
+
+
+# ---------------------------------------------------------------------------------------
+# the CPU oracle (reference arm and the cpu_baseline field)
+# ---------------------------------------------------------------------------------------
+def cpu_baseline(args, n_cols: int | None = None):
+    """The oracle as it stands on a bounded slice of the same layer: the first T_s tokens and the
+    first n_s output features with the full d = 5120 (all six quantized forms, the three GEMMs
+    over every output of the slice)."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    cores = os.cpu_count() or 1
+    T_s = 256
+    n_s = n_cols or min(D_OUT, 1024 * max(1, cores // 8))
+    x = synth.bf16_bits(synth.activations(T_TOK, D_IN, seed=0, outlier_frac=0.001)[:T_s])
+    w = synth.bf16_bits(synth.weights(D_OUT, D_IN, seed=1)[:n_s])
+    dy = synth.bf16_bits(synth.grad_output(T_TOK, D_OUT, seed=2)[:T_s, :n_s])
+    t0 = time.perf_counter()
+    xq = oracle.quantize(x, nthreads=cores)
+    xr = oracle.quantize(x, along=1, rht=True, nthreads=cores)
+    wq = oracle.quantize(w, block=oracle.BLOCK_16x16, nthreads=cores)
+    wqt = oracle.transpose_2d(wq)
+    dq = oracle.quantize(dy, mode=oracle.SR, stream_id=1, nthreads=cores)
+    dr = oracle.quantize(dy, along=1, mode=oracle.SR, rht=True, stream_id=2, nthreads=cores)
+
+    def every(a, b):
+        ii, jj = np.meshgrid(np.arange(a.R), np.arange(b.R), indexing="ij")
+        return oracle.gemm_sampled(a, b, ii.reshape(-1), jj.reshape(-1), nthreads=cores)
+
+    every(xq, wq)
+    every(dq, wqt)
+    every(dr, xr)
+    dt = time.perf_counter() - t0
+    flop = 3 * 2 * T_s * D_IN * n_s
+    return {"value": flop / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "seconds": dt,
+            "sample": f"layer slice T={T_s} tokens x n={n_s} out-features x d={D_IN}: six quantized forms and the "
+                      f"fprop/dgrad/wgrad GEMMs (fp64 over dequantized operands) of the slice, {flop / 1e9:.1f} GFLOP"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline(args, n_cols=256)
+    for _ in range(args.steps):
+        samples.append(cpu_baseline(args, n_cols=256))
+    value = statistics.mean(s["value"] for s in samples)
+    sec = statistics.mean(s["seconds"] for s in samples)
+    return {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp64 GEMM over dequantized NVFP4 operands (CPU)", "data": "synthetic",
+            "config": {"workload": "NVFP4 linear fwd+bwd, bounded slice of T=8192 d=5120 n=20480 (see cpu_baseline)"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": samples[0]["cores"], "kind": "oracle",
+                             "sample": samples[0]["sample"]},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    if rank != 0:
+        args.cpu_baseline = False
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
