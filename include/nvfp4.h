@@ -190,6 +190,22 @@ nvfp4_status nvfp4_gelu_fwd(const void* h, void* g, int64_t n, nvfp4_stream_t st
 nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n,
                             nvfp4_stream_t stream);
 
+/*
+ * nvfp4_quantize without a workspace argument.  The pages have no counterpart: this exists for
+ * callers that cannot allocate device memory themselves (a host whose own allocator owns all
+ * device memory, or a plugin interface without an allocation hook) and so cannot pass `ws`.
+ * Arguments, shape rules and results are those of nvfp4_quantize; the call allocates nothing.
+ * Its 256-byte scratch is a fixed device array inside the library, held by every GPU that
+ * loads the library until the process exits; a call whose scratch would not fit returns
+ * NVFP4_ERR_LIMIT.  The first call on a device looks up the array's device address (do it
+ * before any stream capture).  All calls share the array, so calls that overlap on the GPU
+ * race; serialise them.  Non-finite inputs are not reported by this variant.
+ */
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along,
+                                    nvfp4_round mode, nvfp4_block block, int rht, uint64_t rht_seed,
+                                    uint64_t sr_seed, uint32_t stream_id, nvfp4_tensor* out,
+                                    nvfp4_stream_t stream);
+
 /* Synchronize `stream`, then report (and clear) the device flags of `ws`: NVFP4_ERR_TIMEOUT
  * takes precedence over NVFP4_ERR_NONFINITE; NVFP4_OK when neither is set. */
 nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream);

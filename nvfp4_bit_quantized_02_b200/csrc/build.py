@@ -20,6 +20,7 @@ SOURCES = {
     "api.cu": ["-fmad=false"],
     "gemm_sm100.cu": [],
     "glue.cu": [],
+    "noalloc.cu": [],
 }
 HEADERS = ["nvfp4_device.cuh", "nvfp4_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
