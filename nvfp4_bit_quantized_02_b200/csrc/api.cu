@@ -153,6 +153,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
     p.block16 = b16 ? 1 : 0;
     p.signs = signs;
     p.sr_seed = sr_seed;
+    p.flags = &w->flags;
     if (along == 0) {
         p.codes_row = out->codes;
         p.scales_row = out->scales;
@@ -216,6 +217,7 @@ nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int6
     p.ld = ldx;
     p.signs = signs;
     p.sr_seed = sr_seed;
+    p.flags = &w->flags;
     p.codes_row = out_row->codes;
     p.scales_row = out_row->scales;
     p.st_row = out_row->tensor_scale;
@@ -272,6 +274,7 @@ nvfp4_status nvfp4_quantize_weight(const void* wp, int64_t rows, int64_t cols, i
     p.cols = cols;
     p.ld = ldw;
     p.block16 = 1;
+    p.flags = &w->flags;
     p.codes_row = w_q->codes;
     p.scales_row = w_q->scales;
     p.tiles_row = w_q->tile_scales;

@@ -56,15 +56,21 @@ __device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */)
     return (uint32_t)ceilf(__fmul_rn(__uint_as_float(a), 131072.0f));
 }
 
+// The same decision without computing the threshold: with r' = 65535 - r16,
+//   |u| in [1, 6):  r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + 64 r' + 63 carries into
+//                   bit 22, so the code is ((|u|bits + 64 r' + 63) >> 22) - 252 (the code of
+//                   the lower neighbour is (|u|bits >> 22) - 252), capped at 7 (|u| >= 6);
+//   |u| in [.5, 1): likewise with 128 r' + 127 and a carry into bit 23;
+//   |u| in [0, .5): r16 < |u| * 2^17, compared in fp32 (both sides exact).
 __device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
     const uint32_t b = __float_as_uint(u);
-    const uint32_t sign = (b >> 28) & 8u;
     const uint32_t a = b & 0x7FFFFFFFu;
-    if (a >= 0x40C00000u) return sign | 7u;   // |u| >= 6 (and +-inf)
-    uint32_t code;
-    if (a >= 0x3F800000u) code = 2u + 2u * ((a >> 23) - 127u) + ((a >> 22) & 1u);
-    else code = (a >= 0x3F000000u) ? 1u : 0u;
-    return sign | (code + (r16 < e2m1_sr_threshold(a) ? 1u : 0u));
+    const uint32_t rn = r16 ^ 0xFFFFu;
+    const uint32_t hi = min((a + (rn << 6) + (63u - (252u << 22))) >> 22, 7u);
+    const uint32_t mid = (a + (rn << 7) + (127u - (125u << 23))) >> 23;
+    const uint32_t lo = __uint2float_rn(r16) < __fmul_rn(__uint_as_float(a), 131072.0f) ? 1u : 0u;
+    const uint32_t code = a >= 0x3F800000u ? hi : (a >= 0x3F000000u ? mid : lo);
+    return ((b >> 28) & 8u) | code;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -123,13 +129,13 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
                                             uint32_t k0, uint32_t k1) {
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
-        const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
         c0 = n0;
-        c1 = lo1;
         c2 = n2;
-        c3 = lo0;
         k0 += 0x9E3779B9u;
         k1 += 0xBB67AE85u;
     }

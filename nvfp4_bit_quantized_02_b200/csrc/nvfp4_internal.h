@@ -45,6 +45,7 @@ struct QuantParams {
     uint32_t stream_col;
     uint32_t signs;
     uint64_t sr_seed;
+    uint32_t* flags;  // workspace flags (timeout of a tile copy)
 };
 
 cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax,

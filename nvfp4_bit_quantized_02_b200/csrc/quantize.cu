@@ -21,7 +21,9 @@
 //      16x16 tiles (weights) are a lane pair's 16x16 patch; both forms share its scale.
 // The quantize pass walks the tiles in reverse order of the amax pass so its first wave
 // reads what the amax pass left in L2.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 
@@ -159,217 +161,341 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
 }
 
 // ---------------------------------------------------------------------------------------
-// pass 2: the tile quantizer
+// pass 2: the tile quantizer.
+//
+// A persistent CTA of 256 threads walks 64-row x 256-column tiles (in reverse order of the
+// amax pass).  Each tile is brought into shared memory by one 2D TMA copy (double-buffered:
+// the next tile's copy is in flight while this one is processed) and then consumed in phases
+// whose thread mappings each suit one job, so no thread holds more than one 16-element group:
+//   P  (COL form with SR) the Philox fields of the COL form: one call per (row, 8 columns),
+//      stored as 16-bit fields in shared memory;
+//   T  (16x16) the tile scales: 4 threads per 16x16 tile, two shuffles;
+//   R  (ROW form) one thread per 16-byte chunk (row, 8 columns); a 1x16 block is a lane pair
+//      (one shuffle); the Philox call of the chunk (stream_row) is made in place; each lane
+//      stores 4 code bytes (a warp writes 128 contiguous bytes) and every 4 blocks' scales
+//      leave as one 32-bit store;
+//   C  (COL form) one thread per (column, 16-row group): 16 values read down a column of the
+//      tile, optional 16-point RHT, block scale, codes staged in shared memory;
+//   S  (COL form) the staged codes and scales leave as 16-byte (or 8-byte) row segments.
+// Per-CTA tables hold r_b = S_enc / dec(c) for the 127 finite E4M3 codes (one IEEE division
+// each, identical to dividing per block).
 // ---------------------------------------------------------------------------------------
-constexpr int kTileRows = 64;    // 4 warps x 16 rows
-constexpr int kTileCols = 256;   // 32 lanes x 8 columns
-constexpr int kQuantThreads = 128;
+constexpr int kTileRows = 64;
+constexpr int kTileCols = 256;
+constexpr int kQuantThreads = 256;
+constexpr int kTileBytes = kTileRows * kTileCols * 2;        // 32 KiB of bf16
+constexpr int kRandBytes = kTileRows * kTileCols * 2;        // 16-bit field per element
+constexpr int kStageCodeBytes = 4 * kTileCols * 8;           // [group][column] x 8 bytes
+constexpr int kStageScaleBytes = 4 * kTileCols;              // [group][column]
 
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int p) {
-    return p == 0 ? v.x : p == 1 ? v.y : p == 2 ? v.z : v.w;
+struct QuantSmem {
+    // offsets into the dynamic shared memory (all 128-byte aligned)
+    static constexpr int x0 = 0;
+    static constexpr int x1 = kTileBytes;
+    static constexpr int codes = 2 * kTileBytes;
+    static constexpr int scales = codes + kStageCodeBytes;
+    static constexpr int mult_row = scales + kStageScaleBytes;   // 128 floats
+    static constexpr int mult_col = mult_row + 512;              // 128 floats
+    static constexpr int tile_code = mult_col + 512;             // 64 bytes
+    static constexpr int tile_mult = tile_code + 128;            // 64 floats
+    static constexpr int bars = tile_mult + 256;                 // 2 mbarriers + abort flag
+    static constexpr int rand = bars + 128;                      // COL-form SR fields
+    static constexpr int bytes_no_rand = rand;
+    static constexpr int bytes_rand = rand + kRandBytes;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool q_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
-// Encode 8 fp32 values (already multiplied by r_b) with RNE into 8 nibbles, element 0 lowest.
-__device__ __forceinline__ uint32_t encode8_rne(const float (&u)[8]) {
-    return e2m1x2_rne(u[0], u[1]) | (e2m1x2_rne(u[2], u[3]) << 8) | (e2m1x2_rne(u[4], u[5]) << 16) |
-           (e2m1x2_rne(u[6], u[7]) << 24);
+// bounded wait for a TMA tile: false once `budget_ns` has passed
+__device__ __forceinline__ bool q_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+    if (q_try_wait(bar, parity)) return true;
+    uint64_t t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (q_try_wait(bar, parity)) return true;
+        uint64_t t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > budget_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void q_load_tile(uint32_t dst, const CUtensorMap* map, int32_t col, int32_t row, uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"((uint32_t)kTileBytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t e4m3_of_amax(float amax_b, float s_enc) {
+    return e4m3_rne_sat(__fmul_rn(__fdiv_rn(amax_b, 6.0f), s_enc));
 }
 
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(QuantParams p) {
-    // COL staging: codes [256 columns][4 row groups x 8 bytes], scales [256][4]
-    __shared__ __align__(16) uint8_t s_codes[COL ? kTileCols * 32 : 16];
-    __shared__ __align__(16) uint8_t s_scales[COL ? kTileCols * 4 : 16];
+__global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx, QuantParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* s_mult_row = reinterpret_cast<float*>(smem + QuantSmem::mult_row);
+    float* s_mult_col = reinterpret_cast<float*>(smem + QuantSmem::mult_col);
+    uint8_t* s_tile_code = smem + QuantSmem::tile_code;
+    float* s_tile_mult = reinterpret_cast<float*>(smem + QuantSmem::tile_mult);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QuantSmem::bars);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + QuantSmem::bars + 16);
+    uint16_t* s_rand = reinterpret_cast<uint16_t*>(smem + QuantSmem::rand);
+    uint8_t* s_codes = smem + QuantSmem::codes;
+    uint8_t* s_scales = smem + QuantSmem::scales;
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t rows = p.rows, cols = p.cols, ld = p.ld;
+    const int64_t rows = p.rows, cols = p.cols;
     const int64_t ntr = (rows + kTileRows - 1) / kTileRows;
     const int64_t ntc = (cols + kTileCols - 1) / kTileCols;
     const int64_t ntiles = ntr * ntc;
+    const bool sr_row = ROW && p.sr_row, sr_col = COL && p.sr_col, rht = COL && p.rht_col, b16 = p.block16 != 0;
 
-    const float amax_r = __uint_as_float(ROW ? *p.amax_row : 0u);
-    const float amax_c = __uint_as_float(COL ? *p.amax_col : 0u);
-    const float senc_r = encode_scale(amax_r);
-    const float senc_c = encode_scale(amax_c);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        if (ROW) *p.st_row = decode_scale(amax_r);
-        if (COL) *p.st_col = decode_scale(amax_c);
+    const float senc_r = encode_scale(__uint_as_float(ROW ? *p.amax_row : 0u));
+    const float senc_c = encode_scale(__uint_as_float(COL ? *p.amax_col : 0u));
+    if (blockIdx.x == 0 && tid == 0) {
+        if (ROW) *p.st_row = decode_scale(__uint_as_float(*p.amax_row));
+        if (COL) *p.st_col = decode_scale(__uint_as_float(*p.amax_col));
     }
+    if (tid < 128) {
+        const uint32_t c = (uint32_t)tid;
+        if (ROW) s_mult_row[c] = (c == 0 || c == 127) ? 0.0f : __fdiv_rn(senc_r, e4m3_decode(c));
+        if (COL) s_mult_col[c] = (c == 0 || c == 127) ? 0.0f : __fdiv_rn(senc_c, e4m3_decode(c));
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[0])) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[1])) : "memory");
+        *s_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
 
-    for (int64_t it = blockIdx.x; it < ntiles; it += gridDim.x) {
-        const int64_t t = ntiles - 1 - it;  // reverse of the amax pass
-        const int64_t tr = t / ntc, tc = t - tr * ntc;
-        const int64_t r0 = tr * kTileRows + warp * 16;
-        const int64_t c0 = tc * kTileCols + lane * 8;
-        const bool col_ok = c0 < cols;
-        const bool grp_ok = r0 < rows;
+    int64_t it = blockIdx.x;
+    auto tile_rc = [&](int64_t i, int64_t& tr, int64_t& tc) {
+        const int64_t t = ntiles - 1 - i;
+        tr = t / ntc;
+        tc = t - tr * ntc;
+    };
+    if (tid == 0 && it < ntiles) {
+        int64_t tr, tc;
+        tile_rc(it, tr, tc);
+        q_load_tile(smem_addr(smem + QuantSmem::x0), &tmx, (int32_t)(tc * kTileCols), (int32_t)(tr * kTileRows),
+                    smem_addr(&bars[0]));
+    }
+    int issued = (it < ntiles) ? 1 : 0, consumed = 0;
 
-        uint4 v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            v[i] = make_uint4(0u, 0u, 0u, 0u);
-            if (col_ok && r0 + i < rows) v[i] = ldg_stream(p.x + (r0 + i) * ld + c0);
+    for (int local = 0; it < ntiles; it += gridDim.x, ++local) {
+        const int buf = local & 1;
+        int64_t tr, tc;
+        tile_rc(it, tr, tc);
+        // prefetch the next tile into the other buffer (freed by the previous iteration's sync)
+        if (tid == 0 && it + gridDim.x < ntiles) {
+            int64_t nr, nc;
+            tile_rc(it + gridDim.x, nr, nc);
+            q_load_tile(smem_addr(smem + (buf ? QuantSmem::x0 : QuantSmem::x1)), &tmx, (int32_t)(nc * kTileCols),
+                        (int32_t)(nr * kTileRows), smem_addr(&bars[buf ^ 1]));
+            ++issued;
         }
+        // Philox fields of the COL form do not depend on the tile data: make them while the copy lands
+        if (sr_col) {
+#pragma unroll 1
+            for (int j = tid; j < kTileRows * (kTileCols / 8); j += kQuantThreads) {
+                const int r = j >> 5, grp = j & 31;
+                const int64_t gr = tr * kTileRows + r, gc = tc * kTileCols + grp * 8;
+                if (gr < rows && gc < cols) {
+                    const U4 w = sr_words(p.sr_seed, p.stream_col, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
+                    *reinterpret_cast<uint4*>(s_rand + r * kTileCols + grp * 8) = make_uint4(w.x, w.y, w.z, w.w);
+                }
+            }
+        }
+        if (!q_wait(smem_addr(&bars[buf]), (uint32_t)(local >> 1) & 1u, 2000000000ull)) *s_abort = 1u;
+        __syncthreads();
+        if (*s_abort) {
+            if (tid == 0) atomicOr(p.flags, kFlagTimeout);
+            break;
+        }
+        ++consumed;
+        const uint16_t* sx = reinterpret_cast<const uint16_t*>(smem + (buf ? QuantSmem::x1 : QuantSmem::x0));
+        const int64_t r_base = tr * kTileRows, c_base = tc * kTileCols;
 
-        // ---- 16x16 tile scale (weights): max over the lane pair's 16x16 patch --------------
-        BlockScale tile_sc{0u, 0.0f};
-        if (p.block16) {
+        // ---- T: 16x16 tile scales ------------------------------------------------------------
+        if (b16) {
+            const int tile = tid >> 2, q = tid & 3;          // 64 tiles: 4 row groups x 16 column groups
+            const int g = tile >> 4, cg = tile & 15;
             uint32_t m = 0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                m = mag_max2(m, v[i].x);
-                m = mag_max2(m, v[i].y);
-                m = mag_max2(m, v[i].z);
-                m = mag_max2(m, v[i].w);
+            for (int i = 0; i < 4; ++i) {
+                const uint4* rowp = reinterpret_cast<const uint4*>(sx + (g * 16 + q * 4 + i) * kTileCols + cg * 16);
+                const uint4 a = rowp[0], b = rowp[1];
+                m = mag_max2(m, a.x); m = mag_max2(m, a.y); m = mag_max2(m, a.z); m = mag_max2(m, a.w);
+                m = mag_max2(m, b.x); m = mag_max2(m, b.y); m = mag_max2(m, b.z); m = mag_max2(m, b.w);
             }
             m = max(m & 0xFFFFu, m >> 16);
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            // the tile amax is a bf16 magnitude; both forms see the same tensor amax
-            tile_sc = block_scale(__uint_as_float(m << 16), ROW ? senc_r : senc_c);
-            if (col_ok && grp_ok && (lane & 1) == 0) {
-                if (ROW && p.tiles_row) p.tiles_row[(r0 >> 4) * (cols >> 4) + (c0 >> 4)] = (uint8_t)tile_sc.code;
-                if (COL && p.tiles_col) p.tiles_col[(c0 >> 4) * (rows >> 4) + (r0 >> 4)] = (uint8_t)tile_sc.code;
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const uint32_t code = e4m3_of_amax(__uint_as_float(m << 16), ROW ? senc_r : senc_c);
+            if (q == 0) {
+                s_tile_code[tile] = (uint8_t)code;
+                s_tile_mult[tile] = (ROW ? s_mult_row : s_mult_col)[code];
+                const int64_t gr = r_base + g * 16, gc = c_base + cg * 16;
+                if (gr < rows && gc < cols) {
+                    if (ROW && p.tiles_row) p.tiles_row[(gr >> 4) * (cols >> 4) + (gc >> 4)] = (uint8_t)code;
+                    if (COL && p.tiles_col) p.tiles_col[(gc >> 4) * (rows >> 4) + (gr >> 4)] = (uint8_t)code;
+                }
             }
+            __syncthreads();
         }
 
-        // ---- ROW form: K = columns ------------------------------------------------------------
+        // ---- R: the ROW form -------------------------------------------------------------------
         if (ROW) {
-            const int64_t kb = c0 >> 4;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int64_t r = r0 + i;
-                float x8[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t w = word_of(v[i], q);
-                    x8[2 * q] = bf16_lo(w);
-                    x8[2 * q + 1] = bf16_hi(w);
-                }
-                BlockScale sc = tile_sc;
-                if (!p.block16) {
-                    uint32_t m = 0;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) m = mag_max2(m, word_of(v[i], q));
+#pragma unroll 1
+            for (int j = tid; j < kTileRows * (kTileCols / 8); j += kQuantThreads) {
+                const int r = j >> 5, ch = j & 31;              // a warp covers one row, 32 chunks
+                const int64_t gr = r_base + r, gc = c_base + ch * 8;
+                const uint4 v = *reinterpret_cast<const uint4*>(sx + r * kTileCols + ch * 8);
+                uint32_t code;
+                float mult;
+                if (b16) {
+                    const int tile = ((r >> 4) << 4) + (ch >> 1);
+                    code = s_tile_code[tile];
+                    mult = s_tile_mult[tile];
+                } else {
+                    uint32_t m = mag_max2(mag_max2(mag_max2(mag_max2(0u, v.x), v.y), v.z), v.w);
                     m = max(m & 0xFFFFu, m >> 16);
                     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-                    sc = block_scale(__uint_as_float(m << 16), senc_r);
+                    code = e4m3_of_amax(__uint_as_float(m << 16), senc_r);
+                    mult = s_mult_row[code];
                 }
-                float u[8];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t packed = 0;
+                if (sr_row) {
+                    const U4 rw = sr_words(p.sr_seed, p.stream_row, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
+                    const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = __fmul_rn(x8[e], sc.mult);
-                uint32_t packed;
-                if (p.sr_row) {
-                    const uint64_t g = ((uint64_t)r * (uint64_t)cols + (uint64_t)c0) >> 3;
-                    const U4 w = sr_words(p.sr_seed, p.stream_row, g);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    packed = 0;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        packed |= e2m1_sr(u[e], (ws[e >> 1] >> (16 * (e & 1))) & 0xFFFFu) << (4 * e);
+                    for (int q = 0; q < 4; ++q) {
+                        packed |= e2m1_sr(__fmul_rn(bf16_lo(w4[q]), mult), rr[q] & 0xFFFFu) << (8 * q);
+                        packed |= e2m1_sr(__fmul_rn(bf16_hi(w4[q]), mult), rr[q] >> 16) << (8 * q + 4);
+                    }
                 } else {
-                    packed = encode8_rne(u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        packed |= e2m1x2_rne(__fmul_rn(bf16_lo(w4[q]), mult), __fmul_rn(bf16_hi(w4[q]), mult)) << (8 * q);
                 }
-                if (col_ok && r < rows) {
-                    *reinterpret_cast<uint32_t*>(p.codes_row + r * (cols >> 1) + (c0 >> 1)) = packed;
-                    if ((lane & 1) == 0) p.scales_row[scale_offset(r, kb, p.nkt_row)] = (uint8_t)sc.code;
+                // scales of blocks kb..kb+3 (lanes 8a, 8a+2, 8a+4, 8a+6) -> one 32-bit word
+                uint32_t sw = code;
+                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 8;
+                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 4) << 16;
+                const bool ok = gr < rows && gc < cols;
+                if (ok) {
+                    *reinterpret_cast<uint32_t*>(p.codes_row + gr * (cols >> 1) + (gc >> 1)) = packed;
+                    if ((lane & 7) == 0) {
+                        // blocks past `cols` are padding and must read 0
+                        const int64_t kb = gc >> 4;
+                        const int64_t nv64 = (cols >> 4) - kb;
+                        const int nvalid = nv64 < 4 ? (int)nv64 : 4;
+                        const uint32_t keep = nvalid >= 4 ? 0xFFFFFFFFu : ((1u << (8 * nvalid)) - 1u);
+                        *reinterpret_cast<uint32_t*>(p.scales_row + scale_offset(gr, kb, p.nkt_row)) = sw & keep;
+                    }
                 }
             }
         }
 
-        // ---- COL form: K = rows (transposed operand), optional RHT -------------------------
+        // ---- C: the COL form -------------------------------------------------------------------
         if (COL) {
-            U4 rw[16];
-            if (p.sr_col) {
+            if (sr_col) __syncthreads();   // s_rand complete
+#pragma unroll 1
+            for (int j = tid; j < 4 * kTileCols; j += kQuantThreads) {
+                const int c = j & (kTileCols - 1), g = j >> 8;   // a warp covers 32 columns of one group
+                float v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t g = ((uint64_t)(r0 + i) * (uint64_t)cols + (uint64_t)c0) >> 3;
-                    rw[i] = sr_words(p.sr_seed, p.stream_col, g);
-                }
-            }
+                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float((uint32_t)sx[(g * 16 + i) * kTileCols + c] << 16);
+                if (rht) rht16(v, p.signs);
+                uint32_t code;
+                float mult;
+                if (b16) {
+                    const int tile = (g << 4) + (c >> 4);
+                    code = s_tile_code[tile];
+                    mult = s_tile_mult[tile];
+                } else {
+                    float m = 0.0f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float a[16], b[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = word_of(v[i], q);
-                    a[i] = bf16_lo(w);
-                    b[i] = bf16_hi(w);
+                    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+                    code = e4m3_of_amax(m, senc_c);
+                    mult = s_mult_col[code];
                 }
-                if (p.rht_col) {
-                    rht16(a, p.signs);
-                    rht16(b, p.signs);
-                }
-                BlockScale sa = tile_sc, sb = tile_sc;
-                if (!p.block16) {
-                    float ma = 0.0f, mb = 0.0f;
+                uint32_t c0 = 0, c1 = 0;
+                if (sr_col) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        ma = fmaxf(ma, fabsf(a[i]));
-                        mb = fmaxf(mb, fabsf(b[i]));
-                    }
-                    sa = block_scale(ma, senc_c);
-                    sb = block_scale(mb, senc_c);
-                }
-                uint32_t ca0 = 0, ca1 = 0, cb0 = 0, cb1 = 0;
-                if (p.sr_col) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t w = q == 0 ? rw[i].x : q == 1 ? rw[i].y : q == 2 ? rw[i].z : rw[i].w;
-                        const uint32_t na = e2m1_sr(__fmul_rn(a[i], sa.mult), w & 0xFFFFu);
-                        const uint32_t nb = e2m1_sr(__fmul_rn(b[i], sb.mult), w >> 16);
-                        if (i < 8) {
-                            ca0 |= na << (4 * i);
-                            cb0 |= nb << (4 * i);
-                        } else {
-                            ca1 |= na << (4 * (i - 8));
-                            cb1 |= nb << (4 * (i - 8));
-                        }
+                        const uint32_t n = e2m1_sr(__fmul_rn(v[i], mult), s_rand[(g * 16 + i) * kTileCols + c]);
+                        if (i < 8) c0 |= n << (4 * i);
+                        else c1 |= n << (4 * (i - 8));
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        ca0 |= e2m1x2_rne(__fmul_rn(a[2 * j], sa.mult), __fmul_rn(a[2 * j + 1], sa.mult)) << (8 * j);
-                        ca1 |= e2m1x2_rne(__fmul_rn(a[8 + 2 * j], sa.mult), __fmul_rn(a[9 + 2 * j], sa.mult)) << (8 * j);
-                        cb0 |= e2m1x2_rne(__fmul_rn(b[2 * j], sb.mult), __fmul_rn(b[2 * j + 1], sb.mult)) << (8 * j);
-                        cb1 |= e2m1x2_rne(__fmul_rn(b[8 + 2 * j], sb.mult), __fmul_rn(b[9 + 2 * j], sb.mult)) << (8 * j);
+                    for (int q = 0; q < 4; ++q) {
+                        c0 |= e2m1x2_rne(__fmul_rn(v[2 * q], mult), __fmul_rn(v[2 * q + 1], mult)) << (8 * q);
+                        c1 |= e2m1x2_rne(__fmul_rn(v[8 + 2 * q], mult), __fmul_rn(v[9 + 2 * q], mult)) << (8 * q);
                     }
                 }
-                const int cl = lane * 8 + 2 * q;  // local column of `a`; `b` is cl + 1
-                *reinterpret_cast<uint2*>(s_codes + cl * 32 + warp * 8) = make_uint2(ca0, ca1);
-                *reinterpret_cast<uint2*>(s_codes + (cl + 1) * 32 + warp * 8) = make_uint2(cb0, cb1);
-                s_scales[cl * 4 + warp] = grp_ok ? (uint8_t)sa.code : (uint8_t)0;
-                s_scales[(cl + 1) * 4 + warp] = grp_ok ? (uint8_t)sb.code : (uint8_t)0;
+                const bool grp_ok = r_base + g * 16 < rows;
+                *reinterpret_cast<uint2*>(s_codes + (g * kTileCols + c) * 8) = make_uint2(c0, c1);
+                s_scales[g * kTileCols + c] = grp_ok ? (uint8_t)code : (uint8_t)0;
             }
             __syncthreads();
-            // write: form row = column c, K segment = this tile's rows
-            const int64_t rbase = tr * kTileRows;
-            const int64_t cbase = tc * kTileCols;
-            const int64_t rem_groups = (rows - rbase) >> 4;
-            const int ngroups = rem_groups < 4 ? (int)rem_groups : 4;
-            const int64_t kbytes = rows >> 1;  // bytes per form row
+            // ---- S: staged COL codes and scales to global memory ---------------------------------
+            const int64_t rem = (rows - r_base) >> 4;
+            const int ngroups = rem < 4 ? (int)rem : 4;
+            const int64_t kbytes = rows >> 1;
             if ((rows & 31) == 0) {
-                // 16-byte chunks: 256 columns x 2 chunks (ngroups is even unless the tile is ragged)
-                for (int q = threadIdx.x; q < kTileCols * 2; q += kQuantThreads) {
-                    const int cl = q >> 1, half = q & 1;
-                    if (cbase + cl < cols && 2 * half < ngroups)
-                        *reinterpret_cast<uint4*>(p.codes_col + (cbase + cl) * kbytes + (rbase >> 1) + half * 16) =
-                            *reinterpret_cast<const uint4*>(s_codes + cl * 32 + half * 16);
+#pragma unroll 1
+                for (int j = tid; j < 2 * kTileCols; j += kQuantThreads) {
+                    const int c = j >> 1, half = j & 1;
+                    if (c_base + c < cols && 2 * half < ngroups) {
+                        const uint2 lo = *reinterpret_cast<const uint2*>(s_codes + ((2 * half) * kTileCols + c) * 8);
+                        const uint2 hi = *reinterpret_cast<const uint2*>(s_codes + ((2 * half + 1) * kTileCols + c) * 8);
+                        *reinterpret_cast<uint4*>(p.codes_col + (c_base + c) * kbytes + (r_base >> 1) + half * 16) =
+                            make_uint4(lo.x, lo.y, hi.x, hi.y);
+                    }
                 }
             } else {
-                for (int q = threadIdx.x; q < kTileCols * 4; q += kQuantThreads) {
-                    const int cl = q >> 2, g = q & 3;
-                    if (cbase + cl < cols && g < ngroups)
-                        *reinterpret_cast<uint2*>(p.codes_col + (cbase + cl) * kbytes + (rbase >> 1) + g * 8) =
-                            *reinterpret_cast<const uint2*>(s_codes + cl * 32 + g * 8);
+#pragma unroll 1
+                for (int j = tid; j < 4 * kTileCols; j += kQuantThreads) {
+                    const int c = j >> 2, g = j & 3;
+                    if (c_base + c < cols && g < ngroups)
+                        *reinterpret_cast<uint2*>(p.codes_col + (c_base + c) * kbytes + (r_base >> 1) + g * 8) =
+                            *reinterpret_cast<const uint2*>(s_codes + (g * kTileCols + c) * 8);
                 }
             }
-            for (int cl = threadIdx.x; cl < kTileCols; cl += kQuantThreads) {
-                if (cbase + cl < cols)
-                    *reinterpret_cast<uint32_t*>(p.scales_col + scale_offset(cbase + cl, rbase >> 4, p.nkt_col)) =
-                        *reinterpret_cast<const uint32_t*>(s_scales + cl * 4);
+            for (int c = tid; c < kTileCols; c += kQuantThreads) {
+                if (c_base + c < cols) {
+                    const uint32_t w = (uint32_t)s_scales[c] | ((uint32_t)s_scales[kTileCols + c] << 8) |
+                                       ((uint32_t)s_scales[2 * kTileCols + c] << 16) |
+                                       ((uint32_t)s_scales[3 * kTileCols + c] << 24);
+                    *reinterpret_cast<uint32_t*>(p.scales_col + scale_offset(c_base + c, r_base >> 4, p.nkt_col)) = w;
+                }
             }
-            __syncthreads();
         }
+        __syncthreads();   // the buffer, s_rand and the staging areas are free for the next tile
+    }
+    // copies issued but never consumed (only after a timeout) must land before the CTA exits
+    if (tid == 0) {
+        for (int k = consumed; k < issued; ++k) q_wait(smem_addr(&bars[k & 1]), (uint32_t)(k >> 1) & 1u, 2000000000ull);
     }
 }
 
@@ -437,15 +563,48 @@ cudaError_t launch_amax_rht(const uint16_t* x, int64_t rows, int64_t cols, int64
     return cudaGetLastError();
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
 cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
     const int64_t ntiles = ((p.rows + kTileRows - 1) / kTileRows) * ((p.cols + kTileCols - 1) / kTileCols);
     if (ntiles == 0) return cudaSuccess;
     const bool row = p.codes_row != nullptr, col = p.codes_col != nullptr;
-    const int grid = grid_for(ntiles * kQuantThreads, kQuantThreads, 4);
-    if (row && col) quantize_tile_kernel<true, true><<<grid, kQuantThreads, 0, s>>>(p);
-    else if (row) quantize_tile_kernel<true, false><<<grid, kQuantThreads, 0, s>>>(p);
-    else if (col) quantize_tile_kernel<false, true><<<grid, kQuantThreads, 0, s>>>(p);
-    else return cudaErrorInvalidValue;
+    if (!row && !col) return cudaErrorInvalidValue;
+    auto fn = q_encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)p.cols, (cuuint64_t)p.rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(p.ld * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)kTileCols, (cuuint32_t)kTileRows};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(p.x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const bool rand = col && p.sr_col;
+    const int smem = rand ? QuantSmem::bytes_rand : QuantSmem::bytes_no_rand;
+    void (*kern)(const CUtensorMap, QuantParams) =
+        row && col ? quantize_tile_kernel<true, true> : row ? quantize_tile_kernel<true, false> : quantize_tile_kernel<false, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes_rand);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantThreads, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const int grid = (int)(ntiles < cap ? ntiles : cap);
+    kern<<<grid, kQuantThreads, smem, s>>>(map, p);
     return cudaGetLastError();
 }
 

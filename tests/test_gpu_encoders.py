@@ -106,3 +106,31 @@ def test_rht16_matches_oracle_bit_exact():
         got = out.cpu().numpy()
         want = np.stack([oracle.rht16(r, signs) for r in x])
         assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_e2m1_sr_codes_at_every_threshold():
+    # for every fp32 |u| in [0, 6) (and its negative), the device SR encode at the two 16-bit
+    # random values around the oracle's threshold t(u): r = t - 1 must round up (when t > 0),
+    # r = t must not; a monotone decision in r is then pinned completely
+    L = checks()
+    for lo, hi in ((0x00000000, 0x40C00000),):
+        for start in range(lo, hi, CHUNK):
+            n = min(CHUNK, hi - start)
+            x = (np.arange(n, dtype=np.uint64) + np.uint64(start)).astype(np.uint32).view(np.float32)
+            t = _oracle_chunked(oracle.e2m1_sr_threshold, x, np.uint32)
+            for sign in (1.0, -1.0):
+                xs = (x * np.float32(sign)).astype(np.float32)
+                for r in (np.clip(t.astype(np.int64) - 1, 0, 65535).astype(np.uint32), np.minimum(t, 65535).astype(np.uint32)):
+                    xd = torch.from_numpy(xs).cuda()
+                    rd = torch.from_numpy(r.view(np.int32)).cuda()
+                    out = torch.empty(n, dtype=torch.uint8, device="cuda")
+                    assert L.chk_e2m1_sr(ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(rd.data_ptr()), n,
+                                         ctypes.c_void_p(out.data_ptr())) == 0
+                    got = out.cpu().numpy()
+                    want = np.empty(n, np.uint8)
+                    step = 1 << 21
+                    def work(i):
+                        want[i:i + step] = oracle.e2m1_sr(xs[i:i + step], r[i:i + step])
+                    parallel_map(work, range(0, n, step))
+                    bad = np.nonzero(got != want)[0]
+                    assert bad.size == 0, f"u={xs[bad[0]]!r} r={r[bad[0]]}: gpu {got[bad[0]]} oracle {want[bad[0]]}"
