@@ -5,7 +5,8 @@
 // Large Language Models with NVFP4", 2.A; the FP4 GEMMs of the linear layers are the hot
 // spot, brainai.pro "Details techniques").
 //
-// One CTA computes a 128 x 256 output tile (one SM; 1 CTA per SM by shared memory):
+// Persistent: one CTA per SM walks 128 x 256 output tiles (groups of 8 M tiles swept along N,
+// for L2 reuse); the shared-memory ring runs on across tiles:
 //   warp 0      TMA producer: per 256-wide K block, the A tile (128 rows x 128 bytes) and the
 //               B tile (256 x 128 bytes) by cp.async.bulk.tensor with 128-byte swizzle, and the
 //               matching 512-byte scale tiles by cp.async.bulk, into a 4-stage ring;
@@ -13,7 +14,9 @@
 //               (tcgen05.cp 32x128b.warpx4) and issues tcgen05.mma kind::mxf4nvf4
 //               block_scale scale_vec::4X (M=128, N=256, K=64), accumulating in fp32 in TMEM;
 //               tcgen05.commit frees the stage;
-//   warps 2-5   epilogue: tcgen05.ld 32x32b, times s_tA*s_tB, bf16 or fp32 stores.
+//   warps 2-9   epilogue: two warps per TMEM lane quadrant drain the accumulator into registers
+//               (tcgen05.ld 32x32b), release it to the MMA warp, then scale by s_tA*s_tB and
+//               store bf16 or fp32 -- overlapping the next tile's MMAs.
 // TMEM columns: [0, 256) accumulator; per stage s, [256 + 48 s, +16) scales of A (4 columns per
 // 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).
 // Every mbarrier wait is bounded by a %globaltimer budget; on expiry the CTA raises the timeout
@@ -37,7 +40,7 @@ constexpr int kSFBBytes = (kBN / 128) * (kBK / 64) * 512;  // 4096
 constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // 55296 (54 KiB)
 constexpr int kBarrierBytes = 256;
 constexpr int kGemmSmem = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;   // producer, MMA, 8 epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256, kSfColsPerStage = 48;
 
@@ -156,7 +159,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------------
-// the kernel
+// the kernel: persistent, one CTA per SM, static tile schedule
 // ---------------------------------------------------------------------------------------
 struct GemmParams {
     const uint8_t* sfa;
@@ -167,12 +170,25 @@ struct GemmParams {
     int64_t ldd;
     int32_t out_fp32;
     int32_t M, N, K;
-    int32_t nkt;        // ceil(K / 64): 64-wide K steps (= scale tiles per 128-row tile)
-    int32_t num_kb;     // ceil(K / 256): pipeline stages' worth of K
+    int32_t nkt;            // ceil(K / 64): 64-wide K steps (= scale tiles per 128-row tile)
+    int32_t num_kb;         // ceil(K / 256): pipeline stages' worth of K per tile
     int32_t sfb_row_tiles;  // ceil(N / 128)
+    int32_t tiles_m, tiles_n;
     uint32_t* flags;
     uint64_t budget_ns;
 };
+
+constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quadrant
+constexpr int kGroupM = 8;                         // L2 raster: 8 M tiles swept along N together
+
+// tile index -> (m tile, n tile): groups of kGroupM M tiles, N-major inside a group
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+    const int per_group = kGroupM * tiles_n;
+    const int g = t / per_group, r = t - g * per_group;
+    const int gm = min(kGroupM, tiles_m - g * kGroupM);
+    tn = r / gm;
+    tm = g * kGroupM + (r - tn * gm);
+}
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
@@ -181,16 +197,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* bar_area = smem + kStages * kStageBytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
     uint64_t* empty_bar = full_bar + kStages;
-    uint64_t* accum_bar = empty_bar + kStages;
-    uint64_t* done_bar = accum_bar + 1;
+    uint64_t* tfull_bar = empty_bar + kStages;     // accumulator ready (MMA -> epilogue)
+    uint64_t* tempty_bar = tfull_bar + 1;          // accumulator drained (epilogue -> MMA)
+    uint64_t* done_bar = tempty_bar + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+    const int ntiles = p.tiles_m * p.tiles_n;
 
-    // zero the scale regions once: a B tile past the last 128-row scale tile is never loaded
-    // and must read as zero scales (its codes are zero-filled by TMA)
     for (int i = threadIdx.x; i < kStages * (kSFABytes + kSFBBytes) / 16; i += kGemmThreads) {
         const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
         reinterpret_cast<uint4*>(smem + s * kStageBytes + kABytes + kBBytes)[o] = make_uint4(0, 0, 0, 0);
@@ -200,7 +215,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
-        mbar_init(smem_u32(accum_bar), 1);
+        mbar_init(smem_u32(tfull_bar), 1);
+        mbar_init(smem_u32(tempty_bar), kEpiWarps);
         mbar_init(smem_u32(done_bar), 1);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -222,34 +238,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-            const int rt_a = m0 >> 7;
-            int issued = 0;
-            for (int kb = 0; kb < p.num_kb; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-                if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
-                const int steps = min(4, p.nkt - 4 * kb);
-                const uint32_t sf_bytes = (uint32_t)steps * 512u;
-                int btiles = 0;
-                for (int t = 0; t < 2; ++t) btiles += ((n0 >> 7) + t < p.sfb_row_tiles) ? 1 : 0;
-                const uint32_t full = smem_u32(&full_bar[s]);
-                mbar_expect_tx(full, (uint32_t)(kABytes + kBBytes) + sf_bytes * (uint32_t)(1 + btiles));
-                uint8_t* st = smem + s * kStageBytes;
-                tma_load_2d(smem_u32(st), &tmA, kb * 128, m0, full);
-                tma_load_2d(smem_u32(st + kABytes), &tmB, kb * 128, n0, full);
-                bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + ((int64_t)rt_a * p.nkt + 4 * kb) * 512, sf_bytes, full);
-                for (int t = 0; t < 2; ++t) {
-                    const int rt = (n0 >> 7) + t;
-                    if (rt < p.sfb_row_tiles)
-                        bulk_load(smem_u32(st + kABytes + kBBytes + kSFABytes + t * 2048),
-                                  p.sfb + ((int64_t)rt * p.nkt + 4 * kb) * 512, sf_bytes, full);
+            int g = 0;   // stages issued, across tiles
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+                const int m0 = tm * kBM, n0 = tn * kBN;
+                for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                    if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, p.flags, p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const int steps = min(4, p.nkt - 4 * kb);
+                    const uint32_t sf_bytes = (uint32_t)steps * 512u;
+                    int btiles = 0;
+                    for (int u = 0; u < 2; ++u) btiles += ((n0 >> 7) + u < p.sfb_row_tiles) ? 1 : 0;
+                    const uint32_t full = smem_u32(&full_bar[s]);
+                    mbar_expect_tx(full, (uint32_t)(kABytes + kBBytes) + sf_bytes * (uint32_t)(1 + btiles));
+                    uint8_t* st = smem + s * kStageBytes;
+                    tma_load_2d(smem_u32(st), &tmA, kb * 128, m0, full);
+                    tma_load_2d(smem_u32(st + kABytes), &tmB, kb * 128, n0, full);
+                    bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + ((int64_t)(m0 >> 7) * p.nkt + 4 * kb) * 512,
+                              sf_bytes, full);
+                    for (int u = 0; u < 2; ++u) {
+                        const int rt = (n0 >> 7) + u;
+                        if (rt < p.sfb_row_tiles)
+                            bulk_load(smem_u32(st + kABytes + kBBytes + kSFABytes + u * 2048),
+                                      p.sfb + ((int64_t)rt * p.nkt + 4 * kb) * 512, sf_bytes, full);
+                    }
                 }
-                ++issued;
             }
             if (*abort_flag) {
                 // drain: every copy this thread issued must land before the CTA exits
-                for (int kb = max(0, issued - kStages); kb < issued; ++kb)
-                    mbar_wait(smem_u32(&full_bar[kb % kStages]), (uint32_t)(kb / kStages) & 1u, abort_flag, p.flags,
+                for (int k = max(0, g - kStages); k < g; ++k)
+                    mbar_wait(smem_u32(&full_bar[k % kStages]), (uint32_t)(k / kStages) & 1u, abort_flag, p.flags,
                               p.budget_ns, false);
             }
         }
@@ -257,51 +281,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ------------------------------- MMA issuer -----------------------------------------
         if (lane == 0) {
             const uint32_t sbase = smem_u32(smem);
-            int kb = 0;
-            for (; kb < p.num_kb; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-                if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) break;
+            int g = 0, local = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
+                // the epilogue must have drained the previous tile's accumulator
+                if (!mbar_wait(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
                 tc_fence_after();
-                const int steps = min(4, p.nkt - 4 * kb);
-                const uint32_t a_s = sbase + s * kStageBytes;
-                const uint32_t b_s = a_s + kABytes;
-                const uint32_t sfa_s = b_s + kBBytes;
-                const uint32_t sfb_s = sfa_s + kSFABytes;
-                const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
-                const uint32_t t_sfb = t_sfa + 16;
-                for (int j = 0; j < steps; ++j) {
-                    tmem_cp_sf(t_sfa + 4 * j, desc_sf_tile(sfa_s + 512 * j));
-                    tmem_cp_sf(t_sfb + 8 * j, desc_sf_tile(sfb_s + 512 * j));
-                    tmem_cp_sf(t_sfb + 8 * j + 4, desc_sf_tile(sfb_s + 2048 + 512 * j));
+                for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                    if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int steps = min(4, p.nkt - 4 * kb);
+                    const uint32_t a_s = sbase + s * kStageBytes;
+                    const uint32_t b_s = a_s + kABytes;
+                    const uint32_t sfa_s = b_s + kBBytes;
+                    const uint32_t sfb_s = sfa_s + kSFABytes;
+                    const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
+                    const uint32_t t_sfb = t_sfa + 16;
+                    for (int j = 0; j < steps; ++j) {
+                        tmem_cp_sf(t_sfa + 4 * j, desc_sf_tile(sfa_s + 512 * j));
+                        tmem_cp_sf(t_sfb + 8 * j, desc_sf_tile(sfb_s + 512 * j));
+                        tmem_cp_sf(t_sfb + 8 * j + 4, desc_sf_tile(sfb_s + 2048 + 512 * j));
+                    }
+                    for (int j = 0; j < steps; ++j) {
+                        mma_nvf4(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), kIdesc, t_sfa + 4 * j,
+                                 t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&empty_bar[s]));
                 }
-                for (int j = 0; j < steps; ++j) {
-                    mma_nvf4(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), kIdesc, t_sfa + 4 * j,
-                             t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
-                }
-                mma_commit(smem_u32(&empty_bar[s]));
+                if (ok) mma_commit(smem_u32(tfull_bar));
             }
-            if (kb == p.num_kb) mma_commit(smem_u32(accum_bar));
             // all MMAs of this thread complete before TMEM may be freed
             mma_commit(smem_u32(done_bar));
             mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
         }
     } else {
-        // ------------------------------- epilogue (warps 2..5) ------------------------------
-        const int q = warp & 3;  // TMEM lane quadrant this warp may read
-        const int row = m0 + q * 32 + lane;
-        const bool ok = mbar_wait(smem_u32(accum_bar), 0u, abort_flag, p.flags, p.budget_ns);
-        __syncwarp();
-        if (__all_sync(0xFFFFFFFFu, ok)) {
+        // ------------------------------- epilogue (warps 2..9) ------------------------------
+        const int ew = warp - 2;
+        const int q = warp & 3;                 // TMEM lane quadrant this warp may read
+        const int colhalf = ew >> 2;            // which 128 of the 256 accumulator columns
+        const float alpha = __fmul_rn(*p.sta, *p.stb);
+        int local = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+            int tm, tn;
+            tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+            const int row = tm * kBM + q * 32 + lane;
+            const bool ok = mbar_wait(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
             tc_fence_after();
-            const float alpha = __fmul_rn(*p.sta, *p.stb);
-#pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-                tmem_ld_wait();
-                const int col0 = n0 + c * 32;
-                if (row < p.M && col0 < p.N) {
+            // drain this warp's 32 rows x 128 columns into registers, then free the accumulator
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r[c]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
+            if (row < p.M) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int col0 = tn * kBN + colhalf * 128 + c * 32;
+                    if (col0 >= p.N) continue;
                     const bool full_chunk = col0 + 32 <= p.N;
                     if (p.out_fp32) {
                         float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
@@ -309,20 +354,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
                                 reinterpret_cast<float4*>(out)[j] = make_float4(
-                                    __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
-                                    __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
+                                    __fmul_rn(__uint_as_float(r[c][4 * j]), alpha), __fmul_rn(__uint_as_float(r[c][4 * j + 1]), alpha),
+                                    __fmul_rn(__uint_as_float(r[c][4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[c][4 * j + 3]), alpha));
                         } else {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
-                                if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+                                if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[c][j]), alpha);
                         }
                     } else {
                         uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
                         uint32_t w[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
-                            float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                            const float lo = __fmul_rn(__uint_as_float(r[c][2 * j]), alpha);
+                            const float hi = __fmul_rn(__uint_as_float(r[c][2 * j + 1]), alpha);
                             uint32_t v;
                             asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
                             w[j] = v;
@@ -406,9 +451,15 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     p.nkt = (int32_t)((K + 63) / 64);
     p.num_kb = (int32_t)((K + kBK - 1) / kBK);
     p.sfb_row_tiles = (int32_t)((N + 127) / 128);
+    p.tiles_m = (int32_t)((M + kBM - 1) / kBM);
+    p.tiles_n = (int32_t)((N + kBN - 1) / kBN);
     p.flags = flags;
     p.budget_ns = budget_ns;
-    dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
+    const int grid = (int)(ntiles < sms ? ntiles : sms);
     gemm_nvf4_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }
