@@ -10,15 +10,21 @@
 //   warp 0      TMA producer: per 256-wide K block, the A tile (128 rows x 128 bytes) and the
 //               B tile (256 x 128 bytes) by cp.async.bulk.tensor with 128-byte swizzle, and the
 //               matching 512-byte scale tiles by cp.async.bulk, into a 4-stage ring;
-//   warp 1      allocates 512 TMEM columns; one thread moves each stage's scales into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues tcgen05.mma kind::mxf4nvf4
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma kind::mxf4nvf4
 //               block_scale scale_vec::4X (M=128, N=256, K=64), accumulating in fp32 in TMEM;
 //               tcgen05.commit frees the stage;
+//   warps 10-13 write each stage's scale tiles from shared memory into TMEM with tcgen05.st
+//               (one warp per TMEM lane quadrant).  Moving the scales with tcgen05.cp instead
+//               costs more tensor-pipe time than the MMAs themselves (measured: 12 copies per
+//               256-wide K block take ~790 cycles and serialise with the 512 cycles of MMAs;
+//               the tcgen05.st path takes ~60 cycles and overlaps them);
 //   warps 2-9   epilogue: two warps per TMEM lane quadrant drain the accumulator into registers
 //               (tcgen05.ld 32x32b), release it to the MMA warp, then scale by s_tA*s_tB and
 //               store bf16 or fp32 -- overlapping the next tile's MMAs.
 // TMEM columns: [0, 256) accumulator; per stage s, [256 + 48 s, +16) scales of A (4 columns per
-// 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).
+// 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).  A stage's
+// scale columns are rewritten only after its smem slot was refilled, i.e. after the MMAs that
+// read them completed (tcgen05.commit -> empty -> producer -> full).
 // Every mbarrier wait is bounded by a %globaltimer budget; on expiry the CTA raises the timeout
 // flag, drains its copies and MMAs (again bounded) and frees its TMEM.
 #include <cuda.h>
@@ -40,7 +46,7 @@ constexpr int kSFBBytes = (kBN / 128) * (kBK / 64) * 512;  // 4096
 constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // 55296 (54 KiB)
 constexpr int kBarrierBytes = 256;
 constexpr int kGemmSmem = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
-constexpr int kGemmThreads = 320;   // producer, MMA, 8 epilogue warps
+constexpr int kGemmThreads = 448;   // producer, MMA, 8 epilogue warps, 4 scale warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256, kSfColsPerStage = 48;
 
@@ -121,16 +127,26 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
            (2ull << 61);
 }
-// descriptor of one 512-byte scale tile for tcgen05.cp 32x128b: 32 rows of 16 bytes, no swizzle,
-// core matrices (8 rows x 16 bytes) contiguous: both byte offsets 128
-__device__ __forceinline__ uint64_t desc_sf_tile(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
-           (1ull << 46);
+// tcgen05.st of 16 / 32 consecutive 32-bit columns of this warp's 32 TMEM lanes
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
     asm volatile(
@@ -179,6 +195,7 @@ struct GemmParams {
 };
 
 constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quadrant
+constexpr int kSfWarps = 4;                        // one warp per TMEM lane quadrant
 constexpr int kGroupM = 8;                         // L2 raster: 8 M tiles swept along N together
 
 // tile index -> (m tile, n tile): groups of kGroupM M tiles, N-major inside a group
@@ -197,7 +214,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* bar_area = smem + kStages * kStageBytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
     uint64_t* empty_bar = full_bar + kStages;
-    uint64_t* tfull_bar = empty_bar + kStages;     // accumulator ready (MMA -> epilogue)
+    uint64_t* sfready_bar = empty_bar + kStages;   // stage's scales written into TMEM (scale warps -> MMA)
+    uint64_t* tfull_bar = sfready_bar + kStages;   // accumulator ready (MMA -> epilogue)
     uint64_t* tempty_bar = tfull_bar + 1;          // accumulator drained (epilogue -> MMA)
     uint64_t* done_bar = tempty_bar + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
@@ -214,6 +232,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
+            mbar_init(smem_u32(&sfready_bar[s]), kSfWarps);
         }
         mbar_init(smem_u32(tfull_bar), 1);
         mbar_init(smem_u32(tempty_bar), kEpiWarps);
@@ -294,19 +313,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait(smem_u32(&sfready_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const int steps = min(4, p.nkt - 4 * kb);
                     const uint32_t a_s = sbase + s * kStageBytes;
                     const uint32_t b_s = a_s + kABytes;
-                    const uint32_t sfa_s = b_s + kBBytes;
-                    const uint32_t sfb_s = sfa_s + kSFABytes;
                     const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
                     const uint32_t t_sfb = t_sfa + 16;
-                    for (int j = 0; j < steps; ++j) {
-                        tmem_cp_sf(t_sfa + 4 * j, desc_sf_tile(sfa_s + 512 * j));
-                        tmem_cp_sf(t_sfb + 8 * j, desc_sf_tile(sfb_s + 512 * j));
-                        tmem_cp_sf(t_sfb + 8 * j + 4, desc_sf_tile(sfb_s + 2048 + 512 * j));
-                    }
                     for (int j = 0; j < steps; ++j) {
                         mma_nvf4(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), kIdesc, t_sfa + 4 * j,
                                  t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
@@ -319,11 +335,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mma_commit(smem_u32(done_bar));
             mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
         }
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ------------------------------- epilogue (warps 2..9) ------------------------------
+        // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 128 columns.  Chunks of
+        // 32 columns are read, scaled, converted and stored; the accumulator is released to the
+        // MMA warp as soon as the last chunk has been read.
         const int ew = warp - 2;
-        const int q = warp & 3;                 // TMEM lane quadrant this warp may read
-        const int colhalf = ew >> 2;            // which 128 of the 256 accumulator columns
+        const int q = warp & 3;
+        const int colhalf = ew >> 2;
         const float alpha = __fmul_rn(*p.sta, *p.stb);
         int local = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
@@ -333,56 +352,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool ok = mbar_wait(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
             tc_fence_after();
-            // drain this warp's 32 rows x 128 columns into registers, then free the accumulator
-            uint32_t r[4][32];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r);
+                tmem_ld_wait();
+                if (c == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
+                }
+                const int col0 = tn * kBN + colhalf * 128 + c * 32;
+                if (row >= p.M || col0 >= p.N) continue;
+                const bool full_chunk = col0 + 32 <= p.N;
+                if (p.out_fp32) {
+                    float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
+                    if (full_chunk) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r[c]);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
-            if (row < p.M) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int col0 = tn * kBN + colhalf * 128 + c * 32;
-                    if (col0 >= p.N) continue;
-                    const bool full_chunk = col0 + 32 <= p.N;
-                    if (p.out_fp32) {
-                        float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
-                        if (full_chunk) {
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                reinterpret_cast<float4*>(out)[j] = make_float4(
-                                    __fmul_rn(__uint_as_float(r[c][4 * j]), alpha), __fmul_rn(__uint_as_float(r[c][4 * j + 1]), alpha),
-                                    __fmul_rn(__uint_as_float(r[c][4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[c][4 * j + 3]), alpha));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[c][j]), alpha);
-                        }
+                        for (int j = 0; j < 8; ++j)
+                            reinterpret_cast<float4*>(out)[j] = make_float4(
+                                __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
                     } else {
-                        uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
-                        uint32_t w[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float lo = __fmul_rn(__uint_as_float(r[c][2 * j]), alpha);
-                            const float hi = __fmul_rn(__uint_as_float(r[c][2 * j + 1]), alpha);
-                            uint32_t v;
-                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
-                            w[j] = v;
-                        }
-                        if (full_chunk) {
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+                    }
+                } else {
+                    uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
+                    uint32_t w[16];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                        } else {
+                    for (int j = 0; j < 16; ++j) {
+                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
+                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                        uint32_t v;
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
+                        w[j] = v;
+                    }
+                    if (full_chunk) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
-                        }
+                        for (int j = 0; j < 4; ++j)
+                            reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
                     }
                 }
+            }
+        }
+    } else {
+        // ------------------------------- scale warps (10..13) -------------------------------
+        // Per stage, each warp writes the stage's block scales into its 32 TMEM lanes in the
+        // layout the block-scaled MMA reads: for 64-wide K step j, the scales of A sit in columns
+        // 4j..4j+3 of the stage's A region and lane i of every quadrant holds the 16-byte line i
+        // of the 512-byte scale tile (rows i, i+32, i+64, i+96); B's two 128-row tiles fill
+        // columns 8j..8j+3 and 8j+4..8j+7 of the B region the same way.
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        int g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+            for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                const bool landed = mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns);
+                if (!__all_sync(0xFFFFFFFFu, landed)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* sfa_s = smem + s * kStageBytes + kABytes + kBBytes;
+                const uint8_t* sfb_s = sfa_s + kSFABytes;
+                uint32_t ra[16], rb[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa_s + 512 * j + 16 * lane);
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb_s + 512 * j + 16 * lane);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb_s + 2048 + 512 * j + 16 * lane);
+                    ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+                    rb[8 * j] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
+                    rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+                }
+                const uint32_t t_sfa = tmem + lane_base + kSfCol0 + s * kSfColsPerStage;
+                tmem_st16(t_sfa, ra);
+                tmem_st32(t_sfa + 16, rb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sfready_bar[s])) : "memory");
             }
         }
     }
