@@ -25,13 +25,15 @@
 // 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).  A stage's
 // scale columns are rewritten only after its smem slot was refilled, i.e. after the MMAs that
 // read them completed (tcgen05.commit -> empty -> producer -> full).
-// Every mbarrier wait is bounded by a %globaltimer budget; on expiry the CTA raises the timeout
+// Every mbarrier wait is bounded by a cycle budget; on expiry the CTA raises the timeout
 // flag, drains its copies and MMAs (again bounded) and frees its TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 
 #include "nvfp4_internal.h"
 
@@ -79,25 +81,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t globaltimer() {
+__device__ __forceinline__ uint64_t cycles() {
     uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
     return t;
 }
 
 // Bounded wait.  Returns false if the CTA aborted (another role timed out) or this wait ran out
 // of its budget (then it raises the abort and the timeout flag).  `honor_abort` = false is used
-// by the drain after an abort, which must still see copies land.
+// by the drain after an abort, which must still see copies land.  The budget is counted in SM
+// cycles (2 per nanosecond, i.e. an upper bound for clocks <= 2 GHz); the cycle counter is read
+// only after a burst of polls, so a wait that succeeds quickly costs no timer read.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                           uint32_t* flags, uint64_t budget_ns, bool honor_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = cycles(), limit = 2 * budget_ns;
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (honor_abort && *abort) return false;
-        if (globaltimer() - t0 > budget_ns) {
+        if (cycles() - t0 > limit) {
             *abort = 1u;
             atomicOr(flags, kFlagTimeout);
             return false;
@@ -189,6 +195,7 @@ struct GemmParams {
     int32_t nkt;            // ceil(K / 64): 64-wide K steps (= scale tiles per 128-row tile)
     int32_t num_kb;         // ceil(K / 256): pipeline stages' worth of K per tile
     int32_t sfb_row_tiles;  // ceil(N / 128)
+    int32_t sfa_row_tiles;  // ceil(M / 128)
     int32_t tiles_m, tiles_n;
     uint32_t* flags;
     uint64_t budget_ns;
@@ -452,6 +459,344 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// 2-SM variant: a cluster of two CTAs on an SM pair computes 256 x 256 output tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64).  CTA r of the pair holds rows
+// [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128) of the B tile, and owns the
+// 128 x 256 accumulator of its A rows.  Per 256-wide K block each SM loads 32 KiB of codes
+// (the 1-SM tile loads 48 KiB), so five stages (with the scales) fit in shared memory.  The leader CTA (rank 0)
+// issues the MMAs; each CTA's TMA loads complete on the leader's full barrier; commits
+// multicast to both CTAs.  Each CTA's block scales (A: its own 128 rows; B: all 256 rows) ride
+// the same ring into its shared memory on a local barrier; its scale warps tcgen05.st them into
+// the stage's TMEM region and arrive on the leader's barrier.  No TMA load uses multicast.
+// ---------------------------------------------------------------------------------------
+constexpr int k2Stages = 5;
+constexpr int k2ABytes = 128 * kBK / 2;                // 16384: this CTA's 128 A rows
+constexpr int k2BBytes = 128 * kBK / 2;                // 16384: this CTA's half of the B tile
+constexpr int k2CodeBytes = k2ABytes + k2BBytes;       // 32768: counted on the leader's full barrier
+constexpr int k2StageBytes = k2CodeBytes + kSFABytes + kSFBBytes;  // + own A scales + all B scales = 38912
+constexpr int k2SfRing = k2Stages;                     // one TMEM scale region per stage
+constexpr int k2Smem = k2Stages * k2StageBytes + kBarrierBytes + 1024;
+constexpr uint32_t k2Idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+static_assert(kSfCol0 + k2SfRing * kSfColsPerStage <= kTmemCols, "TMEM budget (2-SM)");
+static_assert(k2StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the object at `saddr` (a shared::cta address) in CTA `rank`
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, volatile uint32_t* abort, uint32_t* flags,
+                                             uint64_t budget_ns, bool honor_abort = true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+        if (mbar_try_wait_cl(bar, parity)) return true;
+    const uint64_t t0 = cycles(), limit = 2 * budget_ns;
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cl(bar, parity)) return true;
+        if (honor_abort && *abort) return false;
+        if (cycles() - t0 > limit) {
+            *abort = 1u;
+            atomicOr(flags, kFlagTimeout);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// arrive on the barrier at this shared::cta offset in both CTAs of the pair, when this thread's
+// prior tcgen05 operations complete
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_local_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* bar_area = smem + k2Stages * k2StageBytes;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);          // leader: TMA bytes of both CTAs
+    uint64_t* empty_bar = full_bar + k2Stages;                            // both: MMAs of the stage done
+    uint64_t* sfready_bar = empty_bar + k2Stages;                         // leader: scales of both CTAs written
+    uint64_t* sffull_bar = sfready_bar + k2SfRing;                        // both: this CTA's scale bytes landed
+    uint64_t* tfull_bar = sffull_bar + k2Stages;                          // both: accumulator ready
+    uint64_t* tempty_bar = tfull_bar + 1;                                 // leader: both epilogues drained
+    uint64_t* done_bar = tempty_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int ntiles = p.tiles_m * p.tiles_n;   // tiles_m counts 256-row tiles here
+
+    for (int i = threadIdx.x; i < k2Stages * (kSFABytes + kSFBBytes) / 16; i += kGemmThreads) {
+        const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
+        reinterpret_cast<uint4*>(smem + s * k2StageBytes + k2CodeBytes)[o] = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < k2Stages; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int f = 0; f < k2SfRing; ++f) mbar_init(smem_u32(&sfready_bar[f]), 2 * kSfWarps);
+        for (int s = 0; s < k2Stages; ++s) mbar_init(smem_u32(&sffull_bar[s]), 1);
+        mbar_init(smem_u32(tfull_bar), 1);
+        mbar_init(smem_u32(tempty_bar), 2 * kEpiWarps);
+        mbar_init(smem_u32(done_bar), 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();   // barriers of both CTAs initialised, TMEM allocated in both
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------- producer (both CTAs) --------------------------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            int g = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < ntiles; t += npairs) {
+                int tm, tn;
+                tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+                const int m0 = tm * 256 + (int)rank * 128, n0 = tn * kBN + (int)rank * 128;
+                for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                    const int s = g % k2Stages;
+                    const uint32_t ph = (uint32_t)(g / k2Stages) & 1u;
+                    if (!mbar_wait_cl(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, p.flags, p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = map_rank(smem_u32(&full_bar[s]), 0);
+                    if (rank == 0) mbar_expect_tx(smem_u32(&full_bar[s]), 2u * (uint32_t)k2CodeBytes);
+                    uint8_t* st = smem + s * k2StageBytes;
+                    tma_load_2d_pair(smem_u32(st), &tmA, kb * 128, m0, full_leader);
+                    tma_load_2d_pair(smem_u32(st + k2ABytes), &tmB, kb * 128, n0, full_leader);
+                    // this CTA's scale tiles (own A rows, both B row tiles) on a local barrier
+                    const int steps = min(4, p.nkt - 4 * kb);
+                    const uint32_t sf_bytes = (uint32_t)steps * 512u;
+                    const int rta = tm * 2 + (int)rank, rtb = tn * 2;
+                    const uint32_t nsf = (rta < p.sfa_row_tiles ? 1u : 0u) + (rtb < p.sfb_row_tiles ? 1u : 0u) +
+                                         (rtb + 1 < p.sfb_row_tiles ? 1u : 0u);
+                    const uint32_t sff = smem_u32(&sffull_bar[s]);
+                    mbar_expect_tx(sff, sf_bytes * nsf);
+                    if (rta < p.sfa_row_tiles)
+                        bulk_load(smem_u32(st + k2CodeBytes), p.sfa + ((int64_t)rta * p.nkt + 4 * kb) * 512, sf_bytes, sff);
+                    for (int u = 0; u < 2; ++u)
+                        if (rtb + u < p.sfb_row_tiles)
+                            bulk_load(smem_u32(st + k2CodeBytes + kSFABytes + u * 2048),
+                                      p.sfb + ((int64_t)(rtb + u) * p.nkt + 4 * kb) * 512, sf_bytes, sff);
+                }
+            }
+            if (*abort_flag) {
+                for (int k = max(0, g - k2Stages); k < g; ++k) {
+                    if (rank == 0)
+                        mbar_wait_cl(smem_u32(&full_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
+                                     p.budget_ns, false);
+                    mbar_wait_cl(smem_u32(&sffull_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
+                                 p.budget_ns, false);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer (leader only) ----------------------------
+        if (lane == 0 && rank == 0) {
+            const uint32_t sbase = smem_u32(smem);
+            int g = 0, local = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
+                if (!mbar_wait_cl(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                    const int s = g % k2Stages, f = g % k2SfRing;
+                    if (!mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns) ||
+                        !mbar_wait_cl(smem_u32(&sfready_bar[f]), (uint32_t)(g / k2SfRing) & 1u, abort_flag, p.flags, p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int steps = min(4, p.nkt - 4 * kb);
+                    const uint32_t a_s = sbase + s * k2StageBytes;
+                    const uint32_t b_s = a_s + k2ABytes;
+                    const uint32_t t_sfa = tmem + kSfCol0 + f * kSfColsPerStage;
+                    const uint32_t t_sfb = t_sfa + 16;
+                    for (int j = 0; j < steps; ++j)
+                        mma_nvf4_pair(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), k2Idesc, t_sfa + 4 * j,
+                                      t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
+                    mma_commit_pair(smem_u32(&empty_bar[s]));
+                }
+                if (ok) mma_commit_pair(smem_u32(tfull_bar));
+            }
+            mma_commit_local_pair(smem_u32(done_bar));
+            mbar_wait_cl(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+        }
+    } else if (warp < 2 + kEpiWarps) {
+        // ------------------------------- epilogue (both CTAs) --------------------------------
+        const int ew = warp - 2;
+        const int q = warp & 3;
+        const int colhalf = ew >> 2;
+        const float alpha = __fmul_rn(*p.sta, *p.stb);
+        const uint32_t tempty_leader = map_rank(smem_u32(tempty_bar), 0);
+        int local = 0;
+        for (int t = pair; t < ntiles; t += npairs, ++local) {
+            int tm, tn;
+            tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+            const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+            const bool ok = mbar_wait_cl(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r);
+                tmem_ld_wait();
+                if (c == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) arrive_cluster(tempty_leader);
+                }
+                const int col0 = tn * kBN + colhalf * 128 + c * 32;
+                if (row >= p.M || col0 >= p.N) continue;
+                const bool full_chunk = col0 + 32 <= p.N;
+                if (p.out_fp32) {
+                    float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
+                    if (full_chunk) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            reinterpret_cast<float4*>(out)[j] = make_float4(
+                                __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+                    }
+                } else {
+                    uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
+                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
+                        uint32_t v;
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
+                        w[j] = v;
+                    }
+                    if (full_chunk) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------- scale warps (both CTAs) -----------------------------
+        // A stage's TMEM scale region is rewritten only after its smem slot was refilled, i.e.
+        // after the MMAs that read the region completed (commit -> empty -> producer -> sffull).
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        int g = 0;
+        bool ok = true;
+        for (int t = pair; ok && t < ntiles; t += npairs) {
+            for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                const int s = g % k2Stages;
+                const bool landed = mbar_wait_cl(smem_u32(&sffull_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag,
+                                                 p.flags, p.budget_ns);
+                if (!__all_sync(0xFFFFFFFFu, landed)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* sfa_s = smem + s * k2StageBytes + k2CodeBytes;
+                const uint8_t* sfb_s = sfa_s + kSFABytes;
+                uint32_t ra[16], rb[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa_s + 512 * j + 16 * lane);
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb_s + 512 * j + 16 * lane);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb_s + 2048 + 512 * j + 16 * lane);
+                    ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+                    rb[8 * j] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
+                    rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
+                }
+                tc_fence_after();
+                const uint32_t t_sfa = tmem + lane_base + kSfCol0 + s * kSfColsPerStage;
+                tmem_st16(t_sfa, ra);
+                tmem_st32(t_sfa + 16, rb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_cluster(map_rank(smem_u32(&sfready_bar[s]), 0));
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs finished with TMEM, barriers and each other's shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -507,6 +852,7 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     p.nkt = (int32_t)((K + 63) / 64);
     p.num_kb = (int32_t)((K + kBK - 1) / kBK);
     p.sfb_row_tiles = (int32_t)((N + 127) / 128);
+    p.sfa_row_tiles = (int32_t)((M + 127) / 128);
     p.tiles_m = (int32_t)((M + kBM - 1) / kBM);
     p.tiles_n = (int32_t)((N + kBN - 1) / kBN);
     p.flags = flags;
@@ -514,6 +860,24 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // 1-SM tiles by default; NVFP4_GEMM_VARIANT=2sm selects the SM-pair kernel for M >= 256
+    // (read on every call)
+    const char* variant = getenv("NVFP4_GEMM_VARIANT");
+    if (variant && strcmp(variant, "2sm") == 0 && M >= 256 && sms >= 2) {
+        static bool attr2_set = false;
+        if (!attr2_set) {
+            cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
+            if (e != cudaSuccess) return e;
+            attr2_set = true;
+        }
+        CUtensorMap ta2, tb2;
+        if (!make_code_map(&ta2, a_codes, M, K, 128) || !make_code_map(&tb2, b_codes, N, K, 128)) return cudaErrorInvalidValue;
+        p.tiles_m = (int32_t)((M + 255) / 256);
+        const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
+        const int64_t pairs = ntiles < sms / 2 ? ntiles : sms / 2;
+        gemm_nvf4_2sm_kernel<<<(unsigned)(2 * pairs), kGemmThreads, k2Smem, stream>>>(ta2, tb2, p);
+        return cudaGetLastError();
+    }
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     gemm_nvf4_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, p);

@@ -218,18 +218,21 @@ __device__ __forceinline__ bool q_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// bounded wait for a TMA tile: false once `budget_ns` has passed
+// bounded wait for a TMA tile: false once about `budget_ns` has passed (counted in SM cycles, 2
+// per nanosecond; the counter is read only after a burst of polls)
 __device__ __forceinline__ bool q_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    if (q_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+        if (q_try_wait(bar, parity)) return true;
     uint64_t t0;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t0));
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 64; ++i)
             if (q_try_wait(bar, parity)) return true;
         uint64_t t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (t - t0 > budget_ns) return false;
+        asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+        if (t - t0 > 2 * budget_ns) return false;
     }
 }
 

@@ -22,9 +22,16 @@ def _exact_operand(rng, R, K):
     return make_form(R, K, nib, sc, 0.125)
 
 
+@pytest.fixture(params=["1sm", "2sm"])
+def variant(request, monkeypatch):
+    # the library reads NVFP4_GEMM_VARIANT on every call; 2sm applies to M >= 256
+    monkeypatch.setenv("NVFP4_GEMM_VARIANT", request.param)
+    return request.param
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (128, 256, 256), (256, 512, 1024), (384, 256, 512),
-                                   (200, 328, 96), (1, 8, 32), (130, 136, 160)])
-def test_exact_dyadic(M, N, K):
+                                   (200, 328, 96), (1, 8, 32), (130, 136, 160), (512, 384, 2048), (300, 200, 96)])
+def test_exact_dyadic(M, N, K, variant):
     m = nv()
     rng = np.random.default_rng(M * 7 + N * 3 + K)
     a, b = _exact_operand(rng, M, K), _exact_operand(rng, N, K)
@@ -35,7 +42,7 @@ def test_exact_dyadic(M, N, K):
     assert bad.size == 0, f"{len(bad)} differ; first {bad[0].tolist()}: gpu {got[tuple(bad[0])]} ref {ref[tuple(bad[0])]}"
 
 
-def test_one_hot_probes_pin_layout():
+def test_one_hot_probes_pin_layout(variant):
     # A row m has a single nonzero element at k = (37 m) % K with a distinct scale per row;
     # D[m][:] is then that element times column k of B: any error in the nibble order or in
     # the position of a scale shows up as a wrong row
@@ -68,7 +75,7 @@ def test_config1_fprop_256(out):
 
 
 @pytest.mark.parametrize("M,N,K", [(512, 768, 1280), (333, 300, 416), (64, 1024, 2048)])
-def test_random_ragged(M, N, K):
+def test_random_ragged(M, N, K, variant):
     m = nv()
     x = synth.bf16_bits(synth.activations(M, K, seed=M))
     w = synth.bf16_bits(synth.weights(N, K, seed=N))
