@@ -123,6 +123,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                  : "memory");
 }
 
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -305,43 +315,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -----------------------------------------
-        if (lane == 0) {
-            const uint32_t sbase = smem_u32(smem);
-            int g = 0, local = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
-                // the epilogue must have drained the previous tile's accumulator
-                if (!mbar_wait(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
+        // The whole warp runs the loop and waits (warp-uniform control flow keeps the MMA
+        // operands uniform); one elected lane issues the MMAs and commits.
+        const uint32_t sbase = smem_u32(smem);
+        const uint64_t adesc0 = desc_k_sw128(sbase), bdesc0 = desc_k_sw128(sbase + kABytes);
+        int g = 0, local = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
+            // the epilogue must have drained the previous tile's accumulator
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag, p.flags,
+                                                   p.budget_ns)))
+                break;
+            tc_fence_after();
+            for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = (uint32_t)(g / kStages) & 1u;
+                const bool landed = mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns) &&
+                                    mbar_wait(smem_u32(&sfready_bar[s]), ph, abort_flag, p.flags, p.budget_ns);
+                if (!__all_sync(0xFFFFFFFFu, landed)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t ph = (uint32_t)(g / kStages) & 1u;
-                    if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait(smem_u32(&sfready_bar[s]), ph, abort_flag, p.flags, p.budget_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const int steps = min(4, p.nkt - 4 * kb);
-                    const uint32_t a_s = sbase + s * kStageBytes;
-                    const uint32_t b_s = a_s + kABytes;
-                    const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
-                    const uint32_t t_sfb = t_sfa + 16;
-                    for (int j = 0; j < steps; ++j) {
-                        mma_nvf4(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), kIdesc, t_sfa + 4 * j,
-                                 t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
-                    }
+                const int steps = min(4, p.nkt - 4 * kb);
+                // descriptors advance by the stage offset and 32 bytes per K step (address field >> 4)
+                const uint64_t aoff = (uint64_t)((s * kStageBytes) >> 4);
+                const uint32_t t_sfa = tmem + kSfCol0 + s * kSfColsPerStage;
+                if (elect_one()) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (j < steps)
+                            mma_nvf4(tmem, adesc0 + aoff + 2 * j, bdesc0 + aoff + 2 * j, kIdesc, t_sfa + 4 * j,
+                                     t_sfa + 16 + 8 * j, (kb | j) != 0 ? 1u : 0u);
                     mma_commit(smem_u32(&empty_bar[s]));
                 }
-                if (ok) mma_commit(smem_u32(tfull_bar));
+                __syncwarp();
             }
-            // all MMAs of this thread complete before TMEM may be freed
-            mma_commit(smem_u32(done_bar));
-            mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+            if (ok && elect_one()) mma_commit(smem_u32(tfull_bar));
+            __syncwarp();
         }
+        // all MMAs of this warp complete before TMEM may be freed
+        if (elect_one()) mma_commit(smem_u32(done_bar));
+        __syncwarp();
+        mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
     } else if (warp < 2 + kEpiWarps) {
         // ------------------------------- epilogue (warps 2..9) ------------------------------
         // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 128 columns.  Chunks of
