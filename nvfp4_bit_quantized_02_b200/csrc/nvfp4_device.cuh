@@ -56,20 +56,20 @@ __device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */)
     return (uint32_t)ceilf(__fmul_rn(__uint_as_float(a), 131072.0f));
 }
 
-// The same decision without computing the threshold: with r' = 65535 - r16,
-//   |u| in [1, 6):  r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + 64 r' + 63 carries into
-//                   bit 22, so the code is ((|u|bits + 64 r' + 63) >> 22) - 252 (the code of
-//                   the lower neighbour is (|u|bits >> 22) - 252), capped at 7 (|u| >= 6);
-//   |u| in [.5, 1): likewise with 128 r' + 127 and a carry into bit 23;
-//   |u| in [0, .5): r16 < |u| * 2^17, compared in fp32 (both sides exact).
+// The same decision without computing the threshold, on a = min(|u|, 6) (6 itself encodes 7):
+//   a in [1, 6]:   r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + (0x3FFFFF - 64 r16) carries
+//                  into bit 22, so the code is ((bits(a) + 0x3FFFFF - 64 r16) >> 22) - 252 (the
+//                  code of the lower neighbour is (bits(a) >> 22) - 252);
+//   a in [.5, 1):  likewise with 0x7FFFFF - 128 r16 and a carry into bit 23;
+//   a in [0, .5):  r16 < a * 2^17, compared in fp32 (both sides exact).
 __device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
     const uint32_t b = __float_as_uint(u);
-    const uint32_t a = b & 0x7FFFFFFFu;
-    const uint32_t rn = r16 ^ 0xFFFFu;
-    const uint32_t hi = min((a + (rn << 6) + (63u - (252u << 22))) >> 22, 7u);
-    const uint32_t mid = (a + (rn << 7) + (127u - (125u << 23))) >> 23;
-    const uint32_t lo = __uint2float_rn(r16) < __fmul_rn(__uint_as_float(a), 131072.0f) ? 1u : 0u;
-    const uint32_t code = a >= 0x3F800000u ? hi : (a >= 0x3F000000u ? mid : lo);
+    const float af = fminf(fabsf(u), 6.0f);
+    const uint32_t a = __float_as_uint(af);
+    const uint32_t hi = (a + (0x3FFFFFu - (252u << 22)) - (r16 << 6)) >> 22;
+    const uint32_t mid = (a + (0x7FFFFFu - (125u << 23)) - (r16 << 7)) >> 23;
+    const uint32_t lo = __uint2float_rn(r16) < __fmul_rn(af, 131072.0f) ? 1u : 0u;
+    const uint32_t code = af >= 1.0f ? hi : (af >= 0.5f ? mid : lo);
     return ((b >> 28) & 8u) | code;
 }
 
@@ -146,6 +146,37 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
 __device__ __forceinline__ U4 sr_words(uint64_t seed, uint32_t stream_id, uint64_t g) {
     return philox4x32_10((uint32_t)g, (uint32_t)(g >> 32), stream_id, 0u, (uint32_t)seed,
                          (uint32_t)(seed >> 32));
+}
+
+// Philox with the ten round keys of one seed computed once (they depend only on the seed).
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+    PhiloxKeys k;
+    uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        k.k0[r] = a;
+        k.k1[r] = b;
+        a += 0x9E3779B9u;
+        b += 0xBB67AE85u;
+    }
+    return k;
+}
+__device__ __forceinline__ U4 sr_words(const PhiloxKeys& k, uint32_t stream_id, uint64_t g) {
+    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = stream_id, c3 = 0u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k.k0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k.k1[r];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+    }
+    return U4{c0, c1, c2, c3};
 }
 
 // ---------------------------------------------------------------------------------------

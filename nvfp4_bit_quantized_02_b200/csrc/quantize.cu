@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
 // pass 1b: plain amax and amax of the 16-point RHT along rows (one read).  A thread takes a
 // 16-row x 8-column patch; rows % 16 == 0, cols % 8 == 0.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t rows,
+__global__ void __launch_bounds__(256, 2) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                        int64_t cols, int64_t ld, uint32_t signs,
                                                        uint32_t* __restrict__ amax_plain_bits,
                                                        uint32_t* __restrict__ amax_rht_bits,
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
             m = mag_max2(m, v[i].z);
             m = mag_max2(m, v[i].w);
         }
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 4; ++p) {
             float a[16], b[16];
 #pragma unroll
@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
     const int64_t ntc = (cols + kTileCols - 1) / kTileCols;
     const int64_t ntiles = ntr * ntc;
     const bool sr_row = ROW && p.sr_row, sr_col = COL && p.sr_col, rht = COL && p.rht_col, b16 = p.block16 != 0;
+    const PhiloxKeys keys = philox_keys(p.sr_seed);
 
     const float senc_r = encode_scale(__uint_as_float(ROW ? *p.amax_row : 0u));
     const float senc_c = encode_scale(__uint_as_float(COL ? *p.amax_col : 0u));
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 const int r = j >> 5, grp = j & 31;
                 const int64_t gr = tr * kTileRows + r, gc = tc * kTileCols + grp * 8;
                 if (gr < rows && gc < cols) {
-                    const U4 w = sr_words(p.sr_seed, p.stream_col, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
+                    const U4 w = sr_words(keys, p.stream_col, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
                     *reinterpret_cast<uint4*>(s_rand + r * kTileCols + grp * 8) = make_uint4(w.x, w.y, w.z, w.w);
                 }
             }
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t packed = 0;
                 if (sr_row) {
-                    const U4 rw = sr_words(p.sr_seed, p.stream_row, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
+                    const U4 rw = sr_words(keys, p.stream_row, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
                     const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
