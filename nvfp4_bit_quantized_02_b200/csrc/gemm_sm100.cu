@@ -13,14 +13,15 @@
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma kind::mxf4nvf4
 //               block_scale scale_vec::4X (M=128, N=256, K=64), accumulating in fp32 in TMEM;
 //               tcgen05.commit frees the stage;
-//   warps 10-13 write each stage's scale tiles from shared memory into TMEM with tcgen05.st
+//   last 4 warps write each stage's scale tiles from shared memory into TMEM with tcgen05.st
 //               (one warp per TMEM lane quadrant).  Moving the scales with tcgen05.cp instead
 //               costs more tensor-pipe time than the MMAs themselves (measured: 12 copies per
 //               256-wide K block take ~790 cycles and serialise with the 512 cycles of MMAs;
 //               the tcgen05.st path takes ~60 cycles and overlaps them);
-//   warps 2-9   epilogue: two warps per TMEM lane quadrant drain the accumulator into registers
-//               (tcgen05.ld 32x32b), release it to the MMA warp, then scale by s_tA*s_tB and
-//               store bf16 or fp32 -- overlapping the next tile's MMAs.
+//   warps 2-17  epilogue: four warps per TMEM lane quadrant, 64 columns each, read the
+//               accumulator into registers (tcgen05.ld 32x32b), release it to the MMA warp, then
+//               scale by s_tA*s_tB and store bf16 or fp32 -- overlapping the next tile's MMAs
+//               (measured: storing before the release stalled the MMAs ~5000 cycles per tile);
 // TMEM columns: [0, 256) accumulator; per stage s, [256 + 48 s, +16) scales of A (4 columns per
 // 64-wide K step), [+16, +48) scales of B (8 columns per K step: two 128-row tiles).  A stage's
 // scale columns are rewritten only after its smem slot was refilled, i.e. after the MMAs that
@@ -46,9 +47,13 @@ constexpr int kBBytes = kBN * kBK / 2;                 // 32768
 constexpr int kSFABytes = (kBM / 128) * (kBK / 64) * 512;  // 2048
 constexpr int kSFBBytes = (kBN / 128) * (kBK / 64) * 512;  // 4096
 constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;  // 55296 (54 KiB)
-constexpr int kBarrierBytes = 256;
-constexpr int kGemmSmem = kStages * kStageBytes + kBarrierBytes + 1024;  // + alignment slack
-constexpr int kGemmThreads = 448;   // producer, MMA, 8 epilogue warps, 4 scale warps
+constexpr int kBarrierBytes = 512;
+constexpr int kStoreSlots = 2;                         // output staging for the TMA stores
+constexpr int kStoreSlotBytes = 32 * 128;              // 32 rows x 128 bytes, 128-byte swizzle
+constexpr int kGemmSmem = kStages * kStageBytes + kStoreSlots * kStoreSlotBytes + kBarrierBytes + 1024;  // + alignment slack
+static_assert(kGemmSmem <= 232448, "1-SM kernel shared memory");
+constexpr int kGemmThreads = 448;   // SM-pair kernel: producer, MMA, 8 epilogue warps, 4 scale warps
+constexpr int kGemm1Threads = 704;  // 1-SM kernel: producer, MMA, 16 epilogue warps, 4 scale warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256, kSfColsPerStage = 48;
 
@@ -190,6 +195,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// shared -> global tile store by the TMA (clipped at the tensor bounds), in this thread's bulk group
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------------
 // the kernel: persistent, one CTA per SM, static tile schedule
 // ---------------------------------------------------------------------------------------
@@ -211,7 +231,8 @@ struct GemmParams {
     uint64_t budget_ns;
 };
 
-constexpr int kEpiWarps = 8;                       // two warps per TMEM lane quadrant
+constexpr int kEpiWarps = 8;                       // SM-pair kernel: two warps per TMEM lane quadrant
+constexpr int kEpi1Warps = 16;                     // 1-SM kernel: four warps per quadrant, 64 columns each
 constexpr int kSfWarps = 4;                        // one warp per TMEM lane quadrant
 constexpr int kGroupM = 8;                         // L2 raster: 8 M tiles swept along N together
 
@@ -224,24 +245,30 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
     tm = g * kGroupM + (r - tn * gm);
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+__global__ void __launch_bounds__(kGemm1Threads, 1)
+    gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmD, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* bar_area = smem + kStages * kStageBytes;
+    uint8_t* store_area = smem + kStages * kStageBytes;
+    uint8_t* bar_area = store_area + kStoreSlots * kStoreSlotBytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
     uint64_t* empty_bar = full_bar + kStages;
     uint64_t* sfready_bar = empty_bar + kStages;   // stage's scales written into TMEM (scale warps -> MMA)
     uint64_t* tfull_bar = sfready_bar + kStages;   // accumulator ready (MMA -> epilogue)
     uint64_t* tempty_bar = tfull_bar + 1;          // accumulator drained (epilogue -> MMA)
     uint64_t* done_bar = tempty_bar + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    // box b of a tile (b = 2 x epilogue warp + half for fp32, = warp for bf16) may write its store
+    // slot once the box two places earlier has been read by its TMA store: one barrier per box
+    // position, so a waiting warp is never more than one phase ahead of its barrier
+    uint64_t* boxgo_bar = done_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(boxgo_bar + 2 * kEpi1Warps);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = p.tiles_m * p.tiles_n;
 
-    for (int i = threadIdx.x; i < kStages * (kSFABytes + kSFBBytes) / 16; i += kGemmThreads) {
+    for (int i = threadIdx.x; i < kStages * (kSFABytes + kSFBBytes) / 16; i += kGemm1Threads) {
         const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
         reinterpret_cast<uint4*>(smem + s * kStageBytes + kABytes + kBBytes)[o] = make_uint4(0, 0, 0, 0);
     }
@@ -252,8 +279,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(smem_u32(&sfready_bar[s]), kSfWarps);
         }
         mbar_init(smem_u32(tfull_bar), 1);
-        mbar_init(smem_u32(tempty_bar), kEpiWarps);
+        mbar_init(smem_u32(tempty_bar), kEpi1Warps);
         mbar_init(smem_u32(done_bar), 1);
+        for (int k = 0; k < 2 * kEpi1Warps; ++k) mbar_init(smem_u32(&boxgo_bar[k]), 1);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -358,74 +386,92 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (elect_one()) mma_commit(smem_u32(done_bar));
         __syncwarp();
         mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
-    } else if (warp < 2 + kEpiWarps) {
-        // ------------------------------- epilogue (warps 2..9) ------------------------------
-        // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 128 columns.  Chunks of
-        // 32 columns are read, scaled, converted and stored; the accumulator is released to the
-        // MMA warp as soon as the last chunk has been read.
+    } else if (warp < 2 + kEpi1Warps) {
+        // ------------------------------- epilogue (warps 2..17) -----------------------------
+        // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 64 columns.  It reads
+        // both 32-column chunks, releases the accumulator to the MMA warp, then scales and
+        // converts in registers and hands the tile to the TMA: 128-byte-wide boxes (64 bf16 or
+        // 32 fp32 columns x 32 rows) staged in one of two swizzled shared-memory slots, which the
+        // warps take in a fixed order (box b of the tile uses slot b % 2 after box b - 2, the last
+        // two boxes of a tile hand over to the first two of the next).  Plain st.global of the rows
+        // (32 lines per instruction) held up the MMA and scale warps' shared-memory traffic for
+        // thousands of cycles per tile; the TMA store leaves that path nearly idle.
         const int ew = warp - 2;
         const int q = warp & 3;
-        const int colhalf = ew >> 2;
+        const int cq = ew >> 2;                 // which 64 of the 256 accumulator columns
         const float alpha = __fmul_rn(*p.sta, *p.stb);
+        const int nbox = p.out_fp32 ? 2 : 1;
+        const uint32_t swz = (uint32_t)(lane & 7);
         int local = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
             int tm, tn;
             tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
-            const int row = tm * kBM + q * 32 + lane;
-            const bool ok = mbar_wait(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            const bool full = mbar_wait(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
+            if (!__all_sync(0xFFFFFFFFu, full)) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r);
-                tmem_ld_wait();
-                if (c == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
+            uint32_t r[2][32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * 64), r[0]);
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * 64 + 32), r[1]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
+            const int y = tm * kBM + q * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h >= nbox) break;
+                const int nb = kEpi1Warps * nbox;            // boxes per tile (even)
+                const int b = ew * nbox + h;
+                const uint32_t slot = (uint32_t)b & 1u;
+                bool free_ok = true;
+                if (b >= 2 || local > 0)   // the n-th completion of a barrier is waited with parity n & 1
+                    free_ok = mbar_wait(smem_u32(&boxgo_bar[b]), (uint32_t)(b >= 2 ? local : local - 1) & 1u, abort_flag,
+                                        p.flags, p.budget_ns);
+                if (!__all_sync(0xFFFFFFFFu, free_ok)) {
+                    ok = false;
+                    break;
                 }
-                const int col0 = tn * kBN + colhalf * 128 + c * 32;
-                if (row >= p.M || col0 >= p.N) continue;
-                const bool full_chunk = col0 + 32 <= p.N;
+                const uint32_t srow = smem_u32(store_area + slot * kStoreSlotBytes) + (uint32_t)lane * 128u;
+                int x;
                 if (p.out_fp32) {
-                    float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
-                    if (full_chunk) {
+                    x = tn * kBN + cq * 64 + h * 32;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            reinterpret_cast<float4*>(out)[j] = make_float4(
-                                __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(srow + (((uint32_t)c ^ swz) << 4),
+                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c]), alpha)),
+                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 1]), alpha)),
+                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 2]), alpha)),
+                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 3]), alpha)));
                 } else {
-                    uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
-                    uint32_t w[16];
+                    x = tn * kBN + cq * 64;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
-                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
-                        uint32_t v;
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
-                        w[j] = v;
-                    }
-                    if (full_chunk) {
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w[4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                        for (int e = 0; e < 4; ++e) {
+                            const int col = 8 * c + 2 * e;   // 0..62 within the warp's 64 columns
+                            const float lo = __fmul_rn(__uint_as_float(r[col >> 5][col & 31]), alpha);
+                            const float hi = __fmul_rn(__uint_as_float(r[col >> 5][(col & 31) + 1]), alpha);
+                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[e]) : "f"(hi), "f"(lo));
+                        }
+                        st_shared_v4(srow + (((uint32_t)c ^ swz) << 4), w[0], w[1], w[2], w[3]);
                     }
                 }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (x < p.N && y < p.M) tma_store_2d(&tmD, smem_u32(store_area + slot * kStoreSlotBytes), x, y);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&boxgo_bar[(b + 2) % nb])) : "memory");
+                }
+                __syncwarp();
             }
         }
+        if (lane == 0) bulk_wait_all();   // this lane's stores are in global memory before the CTA exits
     } else {
-        // ------------------------------- scale warps (10..13) -------------------------------
+        // ------------------------------- scale warps (18..21) -------------------------------
         // Per stage, each warp writes the stage's block scales into its 32 TMEM lanes in the
         // layout the block-scaled MMA reads: for 64-wide K step j, the scales of A sit in columns
         // 4j..4j+3 of the stage's A region and lane i of every quadrant holds the 16-byte line i
@@ -841,6 +887,22 @@ static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int
     return r == CUDA_SUCCESS;
 }
 
+// 2D map over the output D[M][ldd] (bf16 or fp32), box = 128 bytes x 32 rows, 128-byte swizzle;
+// rows >= M and columns >= N of a box are not written
+static bool make_out_map(CUtensorMap* map, void* d, int64_t M, int64_t N, int64_t ldd, bool fp32) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t esz = fp32 ? 4 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldd * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, d, dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
                              const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                              void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
@@ -896,7 +958,9 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     }
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    gemm_nvf4_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, p);
+    CUtensorMap td;
+    if (!make_out_map(&td, d, M, N, ldd, out_fp32)) return cudaErrorInvalidValue;
+    gemm_nvf4_kernel<<<grid, kGemm1Threads, kGemmSmem, stream>>>(ta, tb, td, p);
     return cudaGetLastError();
 }
 
