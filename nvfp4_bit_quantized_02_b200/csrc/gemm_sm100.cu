@@ -52,8 +52,7 @@ constexpr int kStoreSlots = 2;                         // output staging for the
 constexpr int kStoreSlotBytes = 32 * 128;              // 32 rows x 128 bytes, 128-byte swizzle
 constexpr int kGemmSmem = kStages * kStageBytes + kStoreSlots * kStoreSlotBytes + kBarrierBytes + 1024;  // + alignment slack
 static_assert(kGemmSmem <= 232448, "1-SM kernel shared memory");
-constexpr int kGemmThreads = 448;   // SM-pair kernel: producer, MMA, 8 epilogue warps, 4 scale warps
-constexpr int kGemm1Threads = 704;  // 1-SM kernel: producer, MMA, 16 epilogue warps, 4 scale warps
+constexpr int kGemm1Threads = 704;  // producer, MMA, 16 epilogue warps, 4 scale warps (both kernels)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256, kSfColsPerStage = 48;
 
@@ -227,22 +226,100 @@ struct GemmParams {
     int32_t sfb_row_tiles;  // ceil(N / 128)
     int32_t sfa_row_tiles;  // ceil(M / 128)
     int32_t tiles_m, tiles_n;
+    int32_t group_n;        // raster: 1 = groups of kGroup N tiles sweep all M tiles, 0 = the transpose
     uint32_t* flags;
     uint64_t budget_ns;
 };
 
-constexpr int kEpiWarps = 8;                       // SM-pair kernel: two warps per TMEM lane quadrant
-constexpr int kEpi1Warps = 16;                     // 1-SM kernel: four warps per quadrant, 64 columns each
+constexpr int kEpi1Warps = 16;                     // four warps per TMEM lane quadrant, 64 columns each
 constexpr int kSfWarps = 4;                        // one warp per TMEM lane quadrant
-constexpr int kGroupM = 8;                         // L2 raster: 8 M tiles swept along N together
+constexpr int kGroup = 8;                          // L2 raster: tiles of 8 rows (or columns) of tiles swept together
 
-// tile index -> (m tile, n tile): groups of kGroupM M tiles, N-major inside a group
-__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
-    const int per_group = kGroupM * tiles_n;
-    const int g = t / per_group, r = t - g * per_group;
-    const int gm = min(kGroupM, tiles_m - g * kGroupM);
-    tn = r / gm;
-    tm = g * kGroupM + (r - tn * gm);
+// tile index -> (m tile, n tile).  The output is cut into bands of kGroup tile rows (group_n = 0)
+// or tile columns (group_n = 1); the CTAs walk a band across, column by column (row by row), so
+// the band's tiles of one operand stay in L2 while the other operand is swept.  The host picks the
+// orientation that sweeps the smaller operand; alternate bands sweep in opposite directions so the
+// first tiles of a sweep are the last ones of the previous sweep, still in L2.
+__device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm, int& tn) {
+    const int band_len = p.group_n ? p.tiles_m : p.tiles_n;     // tiles along the sweep
+    const int nbands_dim = p.group_n ? p.tiles_n : p.tiles_m;   // tiles across the bands
+    const int per_band = kGroup * band_len;
+    const int g = t / per_band, r = t - g * per_band;
+    const int w = min(kGroup, nbands_dim - g * kGroup);         // width of this band (last may be narrow)
+    int along = r / w;
+    const int across = g * kGroup + (r - along * w);
+    if (g & 1) along = band_len - 1 - along;
+    if (p.group_n) {
+        tm = along;
+        tn = across;
+    } else {
+        tm = across;
+        tn = along;
+    }
+}
+
+// Writes one epilogue warp's 32 rows x 64 accumulator columns (r: two 32-column chunks of fp32
+// bits) to D through the TMA, scaled by alpha: 128-byte-wide boxes (64 bf16 or 32 fp32 columns x
+// 32 rows) staged in kSlots swizzled 4 KiB shared-memory slots, taken in a fixed order.  Box b of
+// a tile (b = warp for bf16, 2 x warp + half for fp32) uses slot b % kSlots once box b - kSlots
+// has been read by its store; the last boxes of a tile hand over to the first ones of the next.
+// One mbarrier per box position keeps every waiting warp at most one phase ahead of it.  Returns
+// false on abort.
+template <int kSlots>
+__device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, uint8_t* store_area, uint64_t* boxgo_bar,
+                                            const uint32_t (&r)[2][32], int ew, int local, int x0, int y,
+                                            const GemmParams& p, float alpha, volatile uint32_t* abort_flag) {
+    const int lane = threadIdx.x & 31;
+    const int nbox = p.out_fp32 ? 2 : 1;
+    const int nb = kEpi1Warps * nbox;   // boxes per tile, a multiple of kSlots
+    const uint32_t swz = (uint32_t)(lane & 7);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (h >= nbox) break;
+        const int b = ew * nbox + h;
+        const uint32_t slot = (uint32_t)(b % kSlots);
+        bool free_ok = true;
+        if (b >= kSlots || local > 0)   // the n-th completion of a barrier is waited with parity n & 1
+            free_ok = mbar_wait(smem_u32(&boxgo_bar[b]), (uint32_t)(b >= kSlots ? local : local - 1) & 1u, abort_flag,
+                                p.flags, p.budget_ns);
+        if (!__all_sync(0xFFFFFFFFu, free_ok)) return false;
+        const uint32_t sbase = smem_u32(store_area + slot * kStoreSlotBytes);
+        const uint32_t srow = sbase + (uint32_t)lane * 128u;
+        int x;
+        if (p.out_fp32) {
+            x = x0 + h * 32;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(srow + (((uint32_t)c ^ swz) << 4), __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c]), alpha)),
+                             __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 1]), alpha)),
+                             __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 2]), alpha)),
+                             __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 3]), alpha)));
+        } else {
+            x = x0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 8 * c + 2 * e;   // 0..62 within the warp's 64 columns
+                    const float lo = __fmul_rn(__uint_as_float(r[col >> 5][col & 31]), alpha);
+                    const float hi = __fmul_rn(__uint_as_float(r[col >> 5][(col & 31) + 1]), alpha);
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[e]) : "f"(hi), "f"(lo));
+                }
+                st_shared_v4(srow + (((uint32_t)c ^ swz) << 4), w[0], w[1], w[2], w[3]);
+            }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            if (x < p.N && y < p.M) tma_store_2d(tmD, sbase, x, y);
+            bulk_commit();
+            bulk_wait_read_all();
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&boxgo_bar[(b + kSlots) % nb])) : "memory");
+        }
+        __syncwarp();
+    }
+    return true;
 }
 
 __global__ void __launch_bounds__(kGemm1Threads, 1)
@@ -258,10 +335,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     uint64_t* tfull_bar = sfready_bar + kStages;   // accumulator ready (MMA -> epilogue)
     uint64_t* tempty_bar = tfull_bar + 1;          // accumulator drained (epilogue -> MMA)
     uint64_t* done_bar = tempty_bar + 1;
-    // box b of a tile (b = 2 x epilogue warp + half for fp32, = warp for bf16) may write its store
-    // slot once the box two places earlier has been read by its TMA store: one barrier per box
-    // position, so a waiting warp is never more than one phase ahead of its barrier
-    uint64_t* boxgo_bar = done_bar + 1;
+    uint64_t* boxgo_bar = done_bar + 1;            // store slot hand-over, one per box position (store_boxes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(boxgo_bar + 2 * kEpi1Warps);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -306,7 +380,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
             bool ok = true;
             for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
                 int tm, tn;
-                tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+                tile_coords(t, p, tm, tn);
                 const int m0 = tm * kBM, n0 = tn * kBN;
                 for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
                     const int s = g % kStages;
@@ -390,23 +464,18 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         // ------------------------------- epilogue (warps 2..17) -----------------------------
         // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 64 columns.  It reads
         // both 32-column chunks, releases the accumulator to the MMA warp, then scales and
-        // converts in registers and hands the tile to the TMA: 128-byte-wide boxes (64 bf16 or
-        // 32 fp32 columns x 32 rows) staged in one of two swizzled shared-memory slots, which the
-        // warps take in a fixed order (box b of the tile uses slot b % 2 after box b - 2, the last
-        // two boxes of a tile hand over to the first two of the next).  Plain st.global of the rows
+        // converts in registers and hands its boxes to the TMA (store_boxes).  Plain st.global of the rows
         // (32 lines per instruction) held up the MMA and scale warps' shared-memory traffic for
         // thousands of cycles per tile; the TMA store leaves that path nearly idle.
         const int ew = warp - 2;
         const int q = warp & 3;
         const int cq = ew >> 2;                 // which 64 of the 256 accumulator columns
         const float alpha = __fmul_rn(*p.sta, *p.stb);
-        const int nbox = p.out_fp32 ? 2 : 1;
-        const uint32_t swz = (uint32_t)(lane & 7);
         int local = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
             int tm, tn;
-            tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+            tile_coords(t, p, tm, tn);
             const bool full = mbar_wait(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
             if (!__all_sync(0xFFFFFFFFu, full)) break;
             tc_fence_after();
@@ -417,57 +486,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
-            const int y = tm * kBM + q * 32;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                if (h >= nbox) break;
-                const int nb = kEpi1Warps * nbox;            // boxes per tile (even)
-                const int b = ew * nbox + h;
-                const uint32_t slot = (uint32_t)b & 1u;
-                bool free_ok = true;
-                if (b >= 2 || local > 0)   // the n-th completion of a barrier is waited with parity n & 1
-                    free_ok = mbar_wait(smem_u32(&boxgo_bar[b]), (uint32_t)(b >= 2 ? local : local - 1) & 1u, abort_flag,
-                                        p.flags, p.budget_ns);
-                if (!__all_sync(0xFFFFFFFFu, free_ok)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t srow = smem_u32(store_area + slot * kStoreSlotBytes) + (uint32_t)lane * 128u;
-                int x;
-                if (p.out_fp32) {
-                    x = tn * kBN + cq * 64 + h * 32;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        st_shared_v4(srow + (((uint32_t)c ^ swz) << 4),
-                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c]), alpha)),
-                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 1]), alpha)),
-                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 2]), alpha)),
-                                     __float_as_uint(__fmul_rn(__uint_as_float(r[h][4 * c + 3]), alpha)));
-                } else {
-                    x = tn * kBN + cq * 64;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int col = 8 * c + 2 * e;   // 0..62 within the warp's 64 columns
-                            const float lo = __fmul_rn(__uint_as_float(r[col >> 5][col & 31]), alpha);
-                            const float hi = __fmul_rn(__uint_as_float(r[col >> 5][(col & 31) + 1]), alpha);
-                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[e]) : "f"(hi), "f"(lo));
-                        }
-                        st_shared_v4(srow + (((uint32_t)c ^ swz) << 4), w[0], w[1], w[2], w[3]);
-                    }
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (x < p.N && y < p.M) tma_store_2d(&tmD, smem_u32(store_area + slot * kStoreSlotBytes), x, y);
-                    bulk_commit();
-                    bulk_wait_read_all();
-                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&boxgo_bar[(b + 2) % nb])) : "memory");
-                }
-                __syncwarp();
-            }
+            ok = store_boxes<kStoreSlots>(&tmD, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64, tm * kBM + q * 32,
+                                          p, alpha, abort_flag);
         }
         if (lane == 0) bulk_wait_all();   // this lane's stores are in global memory before the CTA exits
     } else {
@@ -537,7 +557,9 @@ constexpr int k2BBytes = 128 * kBK / 2;                // 16384: this CTA's half
 constexpr int k2CodeBytes = k2ABytes + k2BBytes;       // 32768: counted on the leader's full barrier
 constexpr int k2StageBytes = k2CodeBytes + kSFABytes + kSFBBytes;  // + own A scales + all B scales = 38912
 constexpr int k2SfRing = k2Stages;                     // one TMEM scale region per stage
-constexpr int k2Smem = k2Stages * k2StageBytes + kBarrierBytes + 1024;
+constexpr int k2StoreSlots = 8;
+constexpr int k2Smem = k2Stages * k2StageBytes + k2StoreSlots * kStoreSlotBytes + kBarrierBytes + 1024;
+static_assert(k2Smem <= 232448, "SM-pair kernel shared memory");
 constexpr uint32_t k2Idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 static_assert(kSfCol0 + k2SfRing * kSfColsPerStage <= kTmemCols, "TMEM budget (2-SM)");
 static_assert(k2StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
@@ -616,11 +638,13 @@ __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
+    gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmD, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* bar_area = smem + k2Stages * k2StageBytes;
+    uint8_t* store_area = smem + k2Stages * k2StageBytes;
+    uint8_t* bar_area = store_area + k2StoreSlots * kStoreSlotBytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);          // leader: TMA bytes of both CTAs
     uint64_t* empty_bar = full_bar + k2Stages;                            // both: MMAs of the stage done
     uint64_t* sfready_bar = empty_bar + k2Stages;                         // leader: scales of both CTAs written
@@ -628,7 +652,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint64_t* tfull_bar = sffull_bar + k2Stages;                          // both: accumulator ready
     uint64_t* tempty_bar = tfull_bar + 1;                                 // leader: both epilogues drained
     uint64_t* done_bar = tempty_bar + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    uint64_t* boxgo_bar = done_bar + 1;                                   // store slot hand-over (store_boxes)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(boxgo_bar + 2 * kEpi1Warps);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -636,7 +661,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int ntiles = p.tiles_m * p.tiles_n;   // tiles_m counts 256-row tiles here
 
-    for (int i = threadIdx.x; i < k2Stages * (kSFABytes + kSFBBytes) / 16; i += kGemmThreads) {
+    for (int i = threadIdx.x; i < k2Stages * (kSFABytes + kSFBBytes) / 16; i += kGemm1Threads) {
         const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
         reinterpret_cast<uint4*>(smem + s * k2StageBytes + k2CodeBytes)[o] = make_uint4(0, 0, 0, 0);
     }
@@ -649,8 +674,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int f = 0; f < k2SfRing; ++f) mbar_init(smem_u32(&sfready_bar[f]), 2 * kSfWarps);
         for (int s = 0; s < k2Stages; ++s) mbar_init(smem_u32(&sffull_bar[s]), 1);
         mbar_init(smem_u32(tfull_bar), 1);
-        mbar_init(smem_u32(tempty_bar), 2 * kEpiWarps);
+        mbar_init(smem_u32(tempty_bar), 2 * kEpi1Warps);
         mbar_init(smem_u32(done_bar), 1);
+        for (int b = 0; b < 2 * kEpi1Warps; ++b) mbar_init(smem_u32(&boxgo_bar[b]), 1);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -674,7 +700,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (int t = pair; ok && t < ntiles; t += npairs) {
                 int tm, tn;
-                tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
+                tile_coords(t, p, tm, tn);
                 const int m0 = tm * 256 + (int)rank * 128, n0 = tn * kBN + (int)rank * 128;
                 for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
                     const int s = g % k2Stages;
@@ -716,100 +742,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer (leader only) ----------------------------
-        if (lane == 0 && rank == 0) {
+        // As in the 1-SM kernel the whole warp runs the loop and one elected lane issues.
+        if (rank == 0) {
             const uint32_t sbase = smem_u32(smem);
+            const uint64_t adesc0 = desc_k_sw128(sbase), bdesc0 = desc_k_sw128(sbase + k2ABytes);
             int g = 0, local = 0;
             bool ok = true;
             for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
-                if (!mbar_wait_cl(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag, p.flags, p.budget_ns)) break;
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_cl(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag,
+                                                          p.flags, p.budget_ns)))
+                    break;
                 tc_fence_after();
                 for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
                     const int s = g % k2Stages, f = g % k2SfRing;
-                    if (!mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns) ||
-                        !mbar_wait_cl(smem_u32(&sfready_bar[f]), (uint32_t)(g / k2SfRing) & 1u, abort_flag, p.flags, p.budget_ns)) {
+                    const bool landed =
+                        mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns) &&
+                        mbar_wait_cl(smem_u32(&sfready_bar[f]), (uint32_t)(g / k2SfRing) & 1u, abort_flag, p.flags, p.budget_ns);
+                    if (!__all_sync(0xFFFFFFFFu, landed)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int steps = min(4, p.nkt - 4 * kb);
-                    const uint32_t a_s = sbase + s * k2StageBytes;
-                    const uint32_t b_s = a_s + k2ABytes;
+                    const uint64_t aoff = (uint64_t)((s * k2StageBytes) >> 4);
                     const uint32_t t_sfa = tmem + kSfCol0 + f * kSfColsPerStage;
-                    const uint32_t t_sfb = t_sfa + 16;
-                    for (int j = 0; j < steps; ++j)
-                        mma_nvf4_pair(tmem, desc_k_sw128(a_s + 32 * j), desc_k_sw128(b_s + 32 * j), k2Idesc, t_sfa + 4 * j,
-                                      t_sfb + 8 * j, (kb | j) != 0 ? 1u : 0u);
-                    mma_commit_pair(smem_u32(&empty_bar[s]));
+                    if (elect_one()) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (j < steps)
+                                mma_nvf4_pair(tmem, adesc0 + aoff + 2 * j, bdesc0 + aoff + 2 * j, k2Idesc, t_sfa + 4 * j,
+                                              t_sfa + 16 + 8 * j, (kb | j) != 0 ? 1u : 0u);
+                        mma_commit_pair(smem_u32(&empty_bar[s]));
+                    }
+                    __syncwarp();
                 }
-                if (ok) mma_commit_pair(smem_u32(tfull_bar));
+                if (ok && elect_one()) mma_commit_pair(smem_u32(tfull_bar));
+                __syncwarp();
             }
-            mma_commit_local_pair(smem_u32(done_bar));
+            if (elect_one()) mma_commit_local_pair(smem_u32(done_bar));
+            __syncwarp();
             mbar_wait_cl(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
         }
-    } else if (warp < 2 + kEpiWarps) {
+    } else if (warp < 2 + kEpi1Warps) {
         // ------------------------------- epilogue (both CTAs) --------------------------------
+        // As in the 1-SM kernel: 16 warps x 64 columns of this CTA's 128 accumulator rows, TMEM
+        // released (on the leader's barrier) before the TMA stores.
         const int ew = warp - 2;
         const int q = warp & 3;
-        const int colhalf = ew >> 2;
+        const int cq = ew >> 2;
         const float alpha = __fmul_rn(*p.sta, *p.stb);
         const uint32_t tempty_leader = map_rank(smem_u32(tempty_bar), 0);
         int local = 0;
-        for (int t = pair; t < ntiles; t += npairs, ++local) {
+        bool ok = true;
+        for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
             int tm, tn;
-            tile_coords(t, p.tiles_m, p.tiles_n, tm, tn);
-            const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
-            const bool ok = mbar_wait_cl(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            tile_coords(t, p, tm, tn);
+            const bool full = mbar_wait_cl(smem_u32(tfull_bar), (uint32_t)local & 1u, abort_flag, p.flags, p.budget_ns);
+            if (!__all_sync(0xFFFFFFFFu, full)) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(colhalf * 128 + c * 32), r);
-                tmem_ld_wait();
-                if (c == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) arrive_cluster(tempty_leader);
-                }
-                const int col0 = tn * kBN + colhalf * 128 + c * 32;
-                if (row >= p.M || col0 >= p.N) continue;
-                const bool full_chunk = col0 + 32 <= p.N;
-                if (p.out_fp32) {
-                    float* out = reinterpret_cast<float*>(p.d) + (int64_t)row * p.ldd + col0;
-                    if (full_chunk) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            reinterpret_cast<float4*>(out)[j] = make_float4(
-                                __fmul_rn(__uint_as_float(r[4 * j]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) out[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
-                    }
-                } else {
-                    uint16_t* out = reinterpret_cast<uint16_t*>(p.d) + (int64_t)row * p.ldd + col0;
-                    uint32_t w[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), alpha);
-                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), alpha);
-                        uint32_t v;
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
-                        w[j] = v;
-                    }
-                    if (full_chunk) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            reinterpret_cast<uint4*>(out)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) out[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
-                    }
-                }
-            }
+            uint32_t r[2][32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * 64), r[0]);
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * 64 + 32), r[1]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_cluster(tempty_leader);
+            ok = store_boxes<k2StoreSlots>(&tmD, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
+                                           tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag);
         }
+        if (lane == 0) bulk_wait_all();
     } else {
         // ------------------------------- scale warps (both CTAs) -----------------------------
         // A stage's TMEM scale region is rewritten only after its smem slot was refilled, i.e.
@@ -933,6 +934,7 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     p.sfa_row_tiles = (int32_t)((M + 127) / 128);
     p.tiles_m = (int32_t)((M + kBM - 1) / kBM);
     p.tiles_n = (int32_t)((N + kBN - 1) / kBN);
+    p.group_n = (M <= N) ? 1 : 0;   // operands are M x K and N x K: sweep the smaller one
     p.flags = flags;
     p.budget_ns = budget_ns;
     int dev = 0, sms = 148;
@@ -953,7 +955,9 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
         p.tiles_m = (int32_t)((M + 255) / 256);
         const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
         const int64_t pairs = ntiles < sms / 2 ? ntiles : sms / 2;
-        gemm_nvf4_2sm_kernel<<<(unsigned)(2 * pairs), kGemmThreads, k2Smem, stream>>>(ta2, tb2, p);
+        CUtensorMap td2;
+        if (!make_out_map(&td2, d, M, N, ldd, out_fp32)) return cudaErrorInvalidValue;
+        gemm_nvf4_2sm_kernel<<<(unsigned)(2 * pairs), kGemm1Threads, k2Smem, stream>>>(ta2, tb2, td2, p);
         return cudaGetLastError();
     }
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
