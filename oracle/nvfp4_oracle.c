@@ -29,8 +29,10 @@
  *   - RNE ties go to the even code, |u| >= 6 saturates to 6, the sign is kept (-0 -> 0x8);
  *   - SR: f = (|u| - lo) / (hi - lo) (exact in fp32), round up iff r16 < ceil(f * 2^16) where
  *     r16 is a 16-bit field of Philox4x32-10 (Salmon et al., SC'11) keyed by the seed with
- *     counter (g_lo, g_hi, stream_id, 0), g = i / 8, i the element's row-major index in the
- *     source tensor, field (i mod 8) = bits [16*(j&1), +16) of output word j>>1;
+ *     counter (g_lo, g_hi, stream_id, 0), g = i / 8, i the element's row-major index r*K + k
+ *     in the quantized form it belongs to (form row r, position k along K; for a transposed
+ *     form that is source element (k, r)), field j = i mod 8 = bits [16*(j&1), +16) of
+ *     output word j>>1;
  *   - RHT: one 16-sign vector per seed (bit j of word 0 of Philox(ctr=(0,0,3,0), key=seed),
  *     set = -1), v = 0.25 * H16 * (D x) with a fixed 4-stage butterfly h = 1, 2, 4, 8;
  *     transformed values stay fp32; amax_t is taken over the transformed values;
@@ -258,10 +260,10 @@ static float form_value(const ora_qjob* j, int64_t r, int64_t k)
     return ora_bf16_to_f32(j->x[sr * j->ld + sc]);
 }
 
-static uint64_t source_index(const ora_qjob* j, int64_t r, int64_t k)
+/* index of the SR bit field of form element (r, k): its row-major position in the form */
+static uint64_t form_index(const ora_qjob* j, int64_t r, int64_t k)
 {
-    int64_t sr = j->along ? k : r, sc = j->along ? r : k;
-    return (uint64_t)(sr * j->cols + sc);
+    return (uint64_t)(r * j->K + k);
 }
 
 /* swizzled offset of the scale of (form row r, K-block kb) */
@@ -323,7 +325,7 @@ static void encode_rows(ora_qjob* j, int64_t r0, int64_t r1)
                     int64_t k = kb * 16 + t + e;
                     float u = row[k] * rb;
                     if (j->mode == 0) q[e] = ora_e2m1_rne(u);
-                    else q[e] = ora_e2m1_sr(u, ora_sr_bits16(j->sr_seed, j->stream_id, source_index(j, r, k)));
+                    else q[e] = ora_e2m1_sr(u, ora_sr_bits16(j->sr_seed, j->stream_id, form_index(j, r, k)));
                 }
                 j->codes[r * (K / 2) + (kb * 16 + t) / 2] = (uint8_t)(q[0] | (q[1] << 4));
             }

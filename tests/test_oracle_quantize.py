@@ -134,12 +134,51 @@ def test_16x16_transpose_identity(ora):
 
 
 def test_along1_equals_transposed_input(ora):
+    # a form depends only on its own values: quantizing x^T through along=1 equals quantizing a
+    # transposed copy, including the SR bits, which are indexed by the position in the form
     x = _x(64, 96, seed=4)
     for rht in (False, True):
-        a = ora.quantize(x, along=1, rht=rht, rht_seed=17)
-        b = ora.quantize(np.ascontiguousarray(x.T), along=0, rht=rht, rht_seed=17)
-        assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales_sw, b.scales_sw)
-        assert a.s_t == b.s_t
+        for mode in (ora.RNE, ora.SR):
+            a = ora.quantize(x, along=1, mode=mode, rht=rht, rht_seed=17, sr_seed=8, stream_id=2)
+            b = ora.quantize(np.ascontiguousarray(x.T), along=0, mode=mode, rht=rht, rht_seed=17, sr_seed=8, stream_id=2)
+            assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales_sw, b.scales_sw)
+            assert a.s_t == b.s_t
+
+
+def test_sr_bits_indexed_by_form_position(ora):
+    # element (r, k) of a form with K columns rounds with the 16-bit field of index r*K + k: the
+    # code of a value strictly between two grid points is its upper neighbour iff
+    # r16 < ceil(f * 2^16), checked on elements whose u the test rebuilds exactly (scale code
+    # 0x38 = 1.0 needs S_enc = 1, i.e. a tensor amax of 2688)
+    rows, cols = 32, 64
+    rng = np.random.default_rng(12)
+    vals = rng.choice(np.array([0.125, 0.375, 0.75, 1.125, 1.375, 2.25, 2.75, 3.5, 4.5, 5.5], np.float32),
+                      size=(rows, cols))
+    vals = vals * np.where(rng.random((rows, cols)) < 0.5, -1, 1).astype(np.float32)
+    vals[:, ::16] = 6.0                      # every block (along rows or columns) has amax 6 ...
+    vals[::16, :] = 6.0
+    vals[0, 0] = 2688.0                      # ... and the tensor amax makes S_enc = 1: scale 1.0
+    x = (vals.view(np.uint32) >> 16).astype(np.uint16)   # all values are exact in bf16
+    for along in (0, 1):
+        q = ora.quantize(x, along=along, mode=ora.SR, sr_seed=99, stream_id=1)
+        v = vals.T if along else vals
+        R, K = v.shape
+        nib = q.nibbles()
+        idx = np.arange(R * K, dtype=np.uint64)
+        r16 = ora.sr_bits16(99, 1, idx).reshape(R, K)
+        grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+        checked = 0
+        for r in range(R):
+            for k in range(K):
+                if q.scales_rm[r, k // 16] != 0x38 or abs(v[r, k]) >= 6.0:
+                    continue
+                a = abs(float(v[r, k]))
+                lo = np.searchsorted(grid, a, side="right") - 1
+                f = (a - grid[lo]) / (grid[lo + 1] - grid[lo])
+                up = r16[r, k] < np.ceil(f * 65536)
+                assert (nib[r, k] & 7) == lo + (1 if up else 0), (along, r, k)
+                checked += 1
+        assert checked > 500
 
 
 def test_rht_amax_is_over_transformed_values(ora):
