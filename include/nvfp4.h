@@ -98,8 +98,9 @@ nvfp4_status nvfp4_workspace_init(void* ws, nvfp4_stream_t stream);
  * along = 1: the form is x^T (form rows = cols, k = rows) -- the token-major wgrad operands.
  * block: 1x16 along k, or 16x16 tiles (weights).  rht = 1 applies the seeded 16-point RHT
  * along k before anything else (1x16 only).  mode = NVFP4_SR draws one 16-bit Philox field
- * per element: key = sr_seed, counter = (i/8 lo, i/8 hi, stream_id, 0), i = the element's
- * row-major index r*cols + c in x.  The RHT signs are bit j of word 0 of
+ * per element: key = sr_seed, counter = (i/8 lo, i/8 hi, stream_id, 0), field i mod 8, where
+ * i = the element's row-major index in the form (form row * k + position along k: r*cols + c
+ * for along = 0, c*rows + r for along = 1).  The RHT signs are bit j of word 0 of
  * Philox(key = rht_seed, counter = (0, 0, 3, 0)), set = -1.
  * Two passes over x: an amax reduction (over the transformed values when rht = 1) and the
  * quantize pass; tensor scales S_enc = 2688/amax_t, s_t = amax_t/2688 (1 and 1 if amax_t == 0).

@@ -167,15 +167,15 @@ __global__ void __launch_bounds__(256, 2) amax_rht_kernel(const uint16_t* __rest
 // amax pass).  Each tile is brought into shared memory by one 2D TMA copy (double-buffered:
 // the next tile's copy is in flight while this one is processed) and then consumed in phases
 // whose thread mappings each suit one job, so no thread holds more than one 16-element group:
-//   P  (COL form with SR) the Philox fields of the COL form: one call per (row, 8 columns),
-//      stored as 16-bit fields in shared memory;
 //   T  (16x16) the tile scales: 4 threads per 16x16 tile, two shuffles;
 //   R  (ROW form) one thread per 16-byte chunk (row, 8 columns); a 1x16 block is a lane pair
 //      (one shuffle); the Philox call of the chunk (stream_row) is made in place; each lane
 //      stores 4 code bytes (a warp writes 128 contiguous bytes) and every 4 blocks' scales
 //      leave as one 32-bit store;
 //   C  (COL form) one thread per (column, 16-row group): 16 values read down a column of the
-//      tile, optional 16-point RHT, block scale, codes staged in shared memory;
+//      tile, optional 16-point RHT, block scale, codes staged in shared memory.  The SR fields
+//      of a form element are indexed by its position in the form, so the 16 elements of a
+//      COL block are two whole Philox calls made in place;
 //   S  (COL form) the staged codes and scales leave as 16-byte (or 8-byte) row segments.
 // Per-CTA tables hold r_b = S_enc / dec(c) for the 127 finite E4M3 codes (one IEEE division
 // each, identical to dividing per block).
@@ -184,7 +184,6 @@ constexpr int kTileRows = 64;
 constexpr int kTileCols = 256;
 constexpr int kQuantThreads = 256;
 constexpr int kTileBytes = kTileRows * kTileCols * 2;        // 32 KiB of bf16
-constexpr int kRandBytes = kTileRows * kTileCols * 2;        // 16-bit field per element
 constexpr int kStageCodeBytes = 4 * kTileCols * 8;           // [group][column] x 8 bytes
 constexpr int kStageScaleBytes = 4 * kTileCols;              // [group][column]
 
@@ -199,9 +198,7 @@ struct QuantSmem {
     static constexpr int tile_code = mult_col + 512;             // 64 bytes
     static constexpr int tile_mult = tile_code + 128;            // 64 floats
     static constexpr int bars = tile_mult + 256;                 // 2 mbarriers + abort flag
-    static constexpr int rand = bars + 128;                      // COL-form SR fields
-    static constexpr int bytes_no_rand = rand;
-    static constexpr int bytes_rand = rand + kRandBytes;
+    static constexpr int bytes = bars + 128;
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -259,7 +256,6 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
     float* s_tile_mult = reinterpret_cast<float*>(smem + QuantSmem::tile_mult);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QuantSmem::bars);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + QuantSmem::bars + 16);
-    uint16_t* s_rand = reinterpret_cast<uint16_t*>(smem + QuantSmem::rand);
     uint8_t* s_codes = smem + QuantSmem::codes;
     uint8_t* s_scales = smem + QuantSmem::scales;
 
@@ -314,18 +310,6 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
             q_load_tile(smem_addr(smem + (buf ? QuantSmem::x0 : QuantSmem::x1)), &tmx, (int32_t)(nc * kTileCols),
                         (int32_t)(nr * kTileRows), smem_addr(&bars[buf ^ 1]));
             ++issued;
-        }
-        // Philox fields of the COL form do not depend on the tile data: make them while the copy lands
-        if (sr_col) {
-#pragma unroll 1
-            for (int j = tid; j < kTileRows * (kTileCols / 8); j += kQuantThreads) {
-                const int r = j >> 5, grp = j & 31;
-                const int64_t gr = tr * kTileRows + r, gc = tc * kTileCols + grp * 8;
-                if (gr < rows && gc < cols) {
-                    const U4 w = sr_words(keys, p.stream_col, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
-                    *reinterpret_cast<uint4*>(s_rand + r * kTileCols + grp * 8) = make_uint4(w.x, w.y, w.z, w.w);
-                }
-            }
         }
         if (!q_wait(smem_addr(&bars[buf]), (uint32_t)(local >> 1) & 1u, 2000000000ull)) *s_abort = 1u;
         __syncthreads();
@@ -421,7 +405,6 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
 
         // ---- C: the COL form -------------------------------------------------------------------
         if (COL) {
-            if (sr_col) __syncthreads();   // s_rand complete
 #pragma unroll 1
             for (int j = tid; j < 4 * kTileCols; j += kQuantThreads) {
                 const int c = j & (kTileCols - 1), g = j >> 8;   // a warp covers 32 columns of one group
@@ -444,9 +427,16 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 }
                 uint32_t c0 = 0, c1 = 0;
                 if (sr_col) {
+                    // form element (column c, row r) has index c * rows + r; the block's first row is a
+                    // multiple of 16, so its 16 fields are Philox calls i0/8 and i0/8 + 1
+                    const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)rows + (uint64_t)(r_base + g * 16)) >> 3;
+                    const U4 w0 = sr_words(keys, p.stream_col, g0);
+                    const U4 w1 = sr_words(keys, p.stream_col, g0 + 1);
+                    const uint32_t rw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const uint32_t n = e2m1_sr(__fmul_rn(v[i], mult), s_rand[(g * 16 + i) * kTileCols + c]);
+                        const uint32_t r16 = (i & 1) ? (rw[i >> 1] >> 16) : (rw[i >> 1] & 0xFFFFu);
+                        const uint32_t n = e2m1_sr(__fmul_rn(v[i], mult), r16);
                         if (i < 8) c0 |= n << (4 * i);
                         else c1 |= n << (4 * (i - 8));
                     }
@@ -495,7 +485,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 }
             }
         }
-        __syncthreads();   // the buffer, s_rand and the staging areas are free for the next tile
+        __syncthreads();   // the buffer and the staging areas are free for the next tile
     }
     // copies issued but never consumed (only after a timeout) must land before the CTA exits
     if (tid == 0) {
@@ -595,11 +585,10 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const bool rand = col && p.sr_col;
-    const int smem = rand ? QuantSmem::bytes_rand : QuantSmem::bytes_no_rand;
+    const int smem = QuantSmem::bytes;
     void (*kern)(const CUtensorMap, QuantParams) =
         row && col ? quantize_tile_kernel<true, true> : row ? quantize_tile_kernel<true, false> : quantize_tile_kernel<false, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes_rand);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
