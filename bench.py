@@ -12,6 +12,7 @@ on its own batch (weak scaling).  --impl reference times the CPU oracle on this 
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -35,6 +36,21 @@ FLOP_GEMM = 2 * T_TOK * D_IN * D_OUT
 Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+# DRAM bytes (read + write) per GEMM launch, the mean over the fprop, dgrad and wgrad launches
+# of one ncu capture (profiles/gemm_nvf4_kernel_8192x5120x20480.md), valid for the GEMM source
+# it was taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
+GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
+GEMM_TRAFFIC = {"sha256": "02ce90f26be9da2f6ebb79bb68d5f60e691abce59a3daf69089311a08e43e634",
+                "bytes_per_launch": 487.7e6}
+
+
+def gemm_traffic():
+    try:
+        with open(GEMM_SRC, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"] if h == GEMM_TRAFFIC["sha256"] else None
 
 
 def load_peaks():
@@ -253,7 +269,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"},
         "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_kernel", "achieved": achieved,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
-                     "traffic": None,
+                     "traffic": gemm_traffic(),
                      "peak_basis": f"{FP4_OVER_BF16:g} x {peak_kind} sustained bf16 ({peaks['bf16_tflops_sustained']} TF/s)",
                      "per_launch_flop": FLOP_GEMM, "avg_launch_ms": gemm_avg_ms},
         "quantize": {"gbs": q_gbs, "unit": "GB/s", "peak_hbm_gbs": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],

@@ -5,8 +5,9 @@
 // Large Language Models with NVFP4", 2.A; the FP4 GEMMs of the linear layers are the hot
 // spot, brainai.pro "Details techniques").
 //
-// Persistent: one CTA per SM walks 128 x 256 output tiles (groups of 8 M tiles swept along N,
-// for L2 reuse); the shared-memory ring runs on across tiles:
+// Persistent: one CTA per SM walks 128 x 256 output tiles (bands of 8 tile rows or columns that
+// sweep the smaller operand, for L2 reuse: tile_coords); the shared-memory ring runs on across
+// tiles:
 //   warp 0      TMA producer: per 256-wide K block, the A tile (128 rows x 128 bytes) and the
 //               B tile (256 x 128 bytes) by cp.async.bulk.tensor with 128-byte swizzle, and the
 //               matching 512-byte scale tiles by cp.async.bulk, into a 4-stage ring;
