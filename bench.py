@@ -122,6 +122,22 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------
+# cross-rank aggregation (weak scaling: every rank runs the whole layer on its own batch)
+# ---------------------------------------------------------------------------------------
+def reduce_max(x: float, dist, device) -> float:
+    """The maximum of x over all ranks (x itself on one rank)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_tflops(world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank did one layer step in the slowest rank's step time."""
+    return world * FLOP_STEP / (ms_per_step * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------------------
 def make_inputs(device):
@@ -193,12 +209,7 @@ def run_ours(args, rank, world, local_rank):
 
     seg = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(6)] for k in range(args.steps)]
     step_ms = [sum(s) for s in seg]
-    ms_total = sum(step_ms)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total_max = t.item()
-    ms_per_step = ms_total_max / args.steps
+    ms_per_step = reduce_max(sum(step_ms), dist, dev) / args.steps
 
     gemm_ms = [s[i] for s in seg for i in (2, 4, 5)]
     q_ms = sum(s[0] + s[1] + s[3] for s in seg)
@@ -239,11 +250,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step(k)
         e1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if dist:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = te.item() / args.e2e_steps
-        e2e = {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+        e2e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / args.e2e_steps
+        e2e = {"value": job_tflops(world, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW"}
 
@@ -251,7 +259,7 @@ def run_ours(args, rank, world, local_rank):
         return None
     line = {
         "metric": METRIC,
-        "value": world * FLOP_STEP / (ms_per_step * 1e-3) / 1e12,
+        "value": job_tflops(world, ms_per_step),
         "unit": "TFLOPS",
         "n_gpus": world,
         "steps": args.steps,
