@@ -275,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
                    "tokens": T_TOK, "d_in": D_IN, "d_out": D_OUT, "rht": "16-point, wgrad operands",
                    "sr": "Philox4x32-10, dY both forms",
                    "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_kernel", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_2sm_kernel", "achieved": achieved,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
                      "traffic": gemm_traffic(),
                      "peak_basis": f"{FP4_OVER_BF16:g} x {peak_kind} sustained bf16 ({peaks['bf16_tflops_sustained']} TF/s)",

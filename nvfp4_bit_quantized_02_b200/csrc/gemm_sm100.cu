@@ -5,7 +5,11 @@
 // Large Language Models with NVFP4", 2.A; the FP4 GEMMs of the linear layers are the hot
 // spot, brainai.pro "Details techniques").
 //
-// Persistent: one CTA per SM walks 128 x 256 output tiles (bands of 8 tile rows or columns that
+// Two kernels.  For M >= 256 the launcher runs the SM-pair kernel further below (256 x 256 tiles
+// on two SMs: fewer operand bytes per SM per K block, a five-stage ring); the 1-SM kernel here
+// serves smaller M (and every shape under NVFP4_GEMM_VARIANT=1sm).
+//
+// 1-SM kernel.  Persistent: one CTA per SM walks 128 x 256 output tiles (bands of 8 tile rows or columns that
 // sweep the smaller operand, for L2 reuse: tile_coords); the shared-memory ring runs on across
 // tiles:
 //   warp 0      TMA producer: per 256-wide K block, the A tile (128 rows x 128 bytes) and the
@@ -546,11 +550,13 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64).  CTA r of the pair holds rows
 // [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128) of the B tile, and owns the
 // 128 x 256 accumulator of its A rows.  Per 256-wide K block each SM loads 32 KiB of codes
-// (the 1-SM tile loads 48 KiB), so five stages (with the scales) fit in shared memory.  The leader CTA (rank 0)
-// issues the MMAs; each CTA's TMA loads complete on the leader's full barrier; commits
-// multicast to both CTAs.  Each CTA's block scales (A: its own 128 rows; B: all 256 rows) ride
-// the same ring into its shared memory on a local barrier; its scale warps tcgen05.st them into
-// the stage's TMEM region and arrive on the leader's barrier.  No TMA load uses multicast.
+// (the 1-SM tile loads 48 KiB), so five stages (with the scales) fit in shared memory.  Each
+// CTA's block scales (A: its own 128 rows; B: all 256 rows) are 2D TMA boxes of 8-byte elements
+// (one 128-row tile's 4 K steps = 2 KiB per box row).  All of a stage's loads, in both CTAs,
+// complete on the leader's full barrier.  The leader CTA (rank 0) then moves the scales into
+// TMEM with tcgen05.cp.cta_group::2 (each CTA from its own shared memory; in a cta_group::2
+// kernel tcgen05.st from scale warps waits for the pair's queued MMAs, ~1400 cycles a stage)
+// and issues the MMAs; commits multicast to both CTAs.  No TMA load uses multicast.
 // ---------------------------------------------------------------------------------------
 constexpr int k2Stages = 5;
 constexpr int k2ABytes = 128 * kBK / 2;                // 16384: this CTA's 128 A rows
@@ -558,6 +564,7 @@ constexpr int k2BBytes = 128 * kBK / 2;                // 16384: this CTA's half
 constexpr int k2CodeBytes = k2ABytes + k2BBytes;       // 32768: counted on the leader's full barrier
 constexpr int k2StageBytes = k2CodeBytes + kSFABytes + kSFBBytes;  // + own A scales + all B scales = 38912
 constexpr int k2SfRing = k2Stages;                     // one TMEM scale region per stage
+constexpr int k2Threads = 576;                         // producer, MMA, 16 epilogue warps
 constexpr int k2StoreSlots = 8;
 constexpr int k2Smem = k2Stages * k2StageBytes + k2StoreSlots * kStoreSlotBytes + kBarrierBytes + 1024;
 static_assert(k2Smem <= 232448, "SM-pair kernel shared memory");
@@ -635,12 +642,24 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
 __device__ __forceinline__ void mma_commit_local_pair(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
+// shared-memory descriptor of a 512-byte scale tile read by tcgen05.cp 32x128b: no swizzle, the
+// 32 16-byte rows one after another (8-row core matrices 128 bytes apart)
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+           (1ull << 46);
+}
+// one 512-byte scale tile (32 rows x 16 bytes) into 4 TMEM columns of all four lane quadrants,
+// in both CTAs of the pair, each from its own shared memory
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                          const __grid_constant__ CUtensorMap tmD, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -648,9 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
     uint8_t* bar_area = store_area + k2StoreSlots * kStoreSlotBytes;
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);          // leader: TMA bytes of both CTAs
     uint64_t* empty_bar = full_bar + k2Stages;                            // both: MMAs of the stage done
-    uint64_t* sfready_bar = empty_bar + k2Stages;                         // leader: scales of both CTAs written
-    uint64_t* sffull_bar = sfready_bar + k2SfRing;                        // both: this CTA's scale bytes landed
-    uint64_t* tfull_bar = sffull_bar + k2Stages;                          // both: accumulator ready
+    uint64_t* tfull_bar = empty_bar + k2Stages;                           // both: accumulator ready
     uint64_t* tempty_bar = tfull_bar + 1;                                 // leader: both epilogues drained
     uint64_t* done_bar = tempty_bar + 1;
     uint64_t* boxgo_bar = done_bar + 1;                                   // store slot hand-over (store_boxes)
@@ -662,18 +679,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int ntiles = p.tiles_m * p.tiles_n;   // tiles_m counts 256-row tiles here
 
-    for (int i = threadIdx.x; i < k2Stages * (kSFABytes + kSFBBytes) / 16; i += kGemm1Threads) {
-        const int s = i / ((kSFABytes + kSFBBytes) / 16), o = i % ((kSFABytes + kSFBBytes) / 16);
-        reinterpret_cast<uint4*>(smem + s * k2StageBytes + k2CodeBytes)[o] = make_uint4(0, 0, 0, 0);
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int s = 0; s < k2Stages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
-        for (int f = 0; f < k2SfRing; ++f) mbar_init(smem_u32(&sfready_bar[f]), 2 * kSfWarps);
-        for (int s = 0; s < k2Stages; ++s) mbar_init(smem_u32(&sffull_bar[s]), 1);
         mbar_init(smem_u32(tfull_bar), 1);
         mbar_init(smem_u32(tempty_bar), 2 * kEpi1Warps);
         mbar_init(smem_u32(done_bar), 1);
@@ -697,6 +707,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSB)) : "memory");
             int g = 0;
             bool ok = true;
             for (int t = pair; ok && t < ntiles; t += npairs) {
@@ -711,34 +723,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
                         break;
                     }
                     const uint32_t full_leader = map_rank(smem_u32(&full_bar[s]), 0);
-                    if (rank == 0) mbar_expect_tx(smem_u32(&full_bar[s]), 2u * (uint32_t)k2CodeBytes);
+                    if (rank == 0) mbar_expect_tx(smem_u32(&full_bar[s]), 2u * (uint32_t)k2StageBytes);
                     uint8_t* st = smem + s * k2StageBytes;
                     tma_load_2d_pair(smem_u32(st), &tmA, kb * 128, m0, full_leader);
                     tma_load_2d_pair(smem_u32(st + k2ABytes), &tmB, kb * 128, n0, full_leader);
-                    // this CTA's scale tiles (own A rows, both B row tiles) on a local barrier
-                    const int steps = min(4, p.nkt - 4 * kb);
-                    const uint32_t sf_bytes = (uint32_t)steps * 512u;
-                    const int rta = tm * 2 + (int)rank, rtb = tn * 2;
-                    const uint32_t nsf = (rta < p.sfa_row_tiles ? 1u : 0u) + (rtb < p.sfb_row_tiles ? 1u : 0u) +
-                                         (rtb + 1 < p.sfb_row_tiles ? 1u : 0u);
-                    const uint32_t sff = smem_u32(&sffull_bar[s]);
-                    mbar_expect_tx(sff, sf_bytes * nsf);
-                    if (rta < p.sfa_row_tiles)
-                        bulk_load(smem_u32(st + k2CodeBytes), p.sfa + ((int64_t)rta * p.nkt + 4 * kb) * 512, sf_bytes, sff);
-                    for (int u = 0; u < 2; ++u)
-                        if (rtb + u < p.sfb_row_tiles)
-                            bulk_load(smem_u32(st + k2CodeBytes + kSFABytes + u * 2048),
-                                      p.sfb + ((int64_t)(rtb + u) * p.nkt + 4 * kb) * 512, sf_bytes, sff);
+                    // scales: this CTA's A row tile and both B row tiles of the pair tile, 4 K steps
+                    // (2 KiB) per row tile; rows and K steps past the tensor read as zero
+                    tma_load_2d_pair(smem_u32(st + k2CodeBytes), &tmSA, kb * 256, tm * 2 + (int)rank, full_leader);
+                    tma_load_2d_pair(smem_u32(st + k2CodeBytes + kSFABytes), &tmSB, kb * 256, tn * 2, full_leader);
                 }
             }
-            if (*abort_flag) {
-                for (int k = max(0, g - k2Stages); k < g; ++k) {
-                    if (rank == 0)
-                        mbar_wait_cl(smem_u32(&full_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
-                                     p.budget_ns, false);
-                    mbar_wait_cl(smem_u32(&sffull_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
+            if (*abort_flag && rank == 0) {
+                // the leader's barrier counts both CTAs' bytes: the peer's copies land on it too
+                for (int k = max(0, g - k2Stages); k < g; ++k)
+                    mbar_wait_cl(smem_u32(&full_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
                                  p.budget_ns, false);
-                }
             }
         }
     } else if (warp == 1) {
@@ -757,8 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
                 for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
                     const int s = g % k2Stages, f = g % k2SfRing;
                     const bool landed =
-                        mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns) &&
-                        mbar_wait_cl(smem_u32(&sfready_bar[f]), (uint32_t)(g / k2SfRing) & 1u, abort_flag, p.flags, p.budget_ns);
+                        mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns);
                     if (!__all_sync(0xFFFFFFFFu, landed)) {
                         ok = false;
                         break;
@@ -768,6 +766,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
                     const uint64_t aoff = (uint64_t)((s * k2StageBytes) >> 4);
                     const uint32_t t_sfa = tmem + kSfCol0 + f * kSfColsPerStage;
                     if (elect_one()) {
+                        const uint32_t sf_s = sbase + s * k2StageBytes + k2CodeBytes;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (j < steps) {
+                                tmem_cp_sf_pair(t_sfa + 4 * j, desc_sf(sf_s + 512 * j));
+                                tmem_cp_sf_pair(t_sfa + 16 + 8 * j, desc_sf(sf_s + kSFABytes + 512 * j));
+                                tmem_cp_sf_pair(t_sfa + 20 + 8 * j, desc_sf(sf_s + kSFABytes + 2048 + 512 * j));
+                            }
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             if (j < steps)
@@ -812,44 +818,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemm1Threads, 1)
                                            tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag);
         }
         if (lane == 0) bulk_wait_all();
-    } else {
-        // ------------------------------- scale warps (both CTAs) -----------------------------
-        // A stage's TMEM scale region is rewritten only after its smem slot was refilled, i.e.
-        // after the MMAs that read the region completed (commit -> empty -> producer -> sffull).
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        int g = 0;
-        bool ok = true;
-        for (int t = pair; ok && t < ntiles; t += npairs) {
-            for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
-                const int s = g % k2Stages;
-                const bool landed = mbar_wait_cl(smem_u32(&sffull_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag,
-                                                 p.flags, p.budget_ns);
-                if (!__all_sync(0xFFFFFFFFu, landed)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* sfa_s = smem + s * k2StageBytes + k2CodeBytes;
-                const uint8_t* sfb_s = sfa_s + kSFABytes;
-                uint32_t ra[16], rb[32];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(sfa_s + 512 * j + 16 * lane);
-                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb_s + 512 * j + 16 * lane);
-                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb_s + 2048 + 512 * j + 16 * lane);
-                    ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
-                    rb[8 * j] = b0.x; rb[8 * j + 1] = b0.y; rb[8 * j + 2] = b0.z; rb[8 * j + 3] = b0.w;
-                    rb[8 * j + 4] = b1.x; rb[8 * j + 5] = b1.y; rb[8 * j + 6] = b1.z; rb[8 * j + 7] = b1.w;
-                }
-                tc_fence_after();
-                const uint32_t t_sfa = tmem + lane_base + kSfCol0 + s * kSfColsPerStage;
-                tmem_st16(t_sfa, ra);
-                tmem_st32(t_sfa + 16, rb);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) arrive_cluster(map_rank(smem_u32(&sfready_bar[s]), 0));
-            }
-        }
     }
 
     tc_fence_before();
@@ -885,6 +853,21 @@ static bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int
     cuuint32_t estr[2] = {1u, 1u};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2D map over the swizzled scale tiles of a form, in 8-byte elements: row = 128-row tile,
+// nkt x 512 bytes per row; box = 256 elements (the 4 K steps of one 256-wide K block) x box_rows
+static bool make_sf_map(CUtensorMap* map, const void* scales, int64_t row_tiles, int64_t nkt, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(nkt * 64), (cuuint64_t)row_tiles};
+    cuuint64_t strides[1] = {(cuuint64_t)(nkt * 512)};
+    cuuint32_t box[2] = {256u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(scales), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -941,10 +924,11 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // 1-SM tiles by default; NVFP4_GEMM_VARIANT=2sm selects the SM-pair kernel for M >= 256
-    // (read on every call)
+    // SM-pair tiles for M >= 256 (fewer operand bytes per SM per K block, a deeper ring);
+    // NVFP4_GEMM_VARIANT=1sm selects the 1-SM kernel for every shape (read on every call)
     const char* variant = getenv("NVFP4_GEMM_VARIANT");
-    if (variant && strcmp(variant, "2sm") == 0 && M >= 256 && sms >= 2) {
+    const bool force_1sm = variant && strcmp(variant, "1sm") == 0;
+    if (!force_1sm && M >= 256 && sms >= 2) {
         static bool attr2_set = false;
         if (!attr2_set) {
             cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
@@ -956,9 +940,11 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
         p.tiles_m = (int32_t)((M + 255) / 256);
         const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
         const int64_t pairs = ntiles < sms / 2 ? ntiles : sms / 2;
-        CUtensorMap td2;
-        if (!make_out_map(&td2, d, M, N, ldd, out_fp32)) return cudaErrorInvalidValue;
-        gemm_nvf4_2sm_kernel<<<(unsigned)(2 * pairs), kGemm1Threads, k2Smem, stream>>>(ta2, tb2, td2, p);
+        CUtensorMap td2, tsa, tsb;
+        if (!make_out_map(&td2, d, M, N, ldd, out_fp32) || !make_sf_map(&tsa, a_scales, p.sfa_row_tiles, p.nkt, 1) ||
+            !make_sf_map(&tsb, b_scales, p.sfb_row_tiles, p.nkt, 2))
+            return cudaErrorInvalidValue;
+        gemm_nvf4_2sm_kernel<<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2, p);
         return cudaGetLastError();
     }
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;

@@ -24,7 +24,8 @@ def _exact_operand(rng, R, K):
 
 @pytest.fixture(params=["1sm", "2sm"])
 def variant(request, monkeypatch):
-    # the library reads NVFP4_GEMM_VARIANT on every call; 2sm applies to M >= 256
+    # the library reads NVFP4_GEMM_VARIANT on every call: 1sm forces the 1-SM kernel; otherwise
+    # the SM-pair kernel runs for M >= 256 and the 1-SM kernel below that
     monkeypatch.setenv("NVFP4_GEMM_VARIANT", request.param)
     return request.param
 
