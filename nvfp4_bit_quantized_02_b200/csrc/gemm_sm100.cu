@@ -583,8 +583,11 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
+// arrive on an mbarrier of the other CTA of the pair.  The default (.release at .cta scope) form:
+// what crosses the pair here is the completion of tcgen05 work, ordered by the tcgen05 fences
+// around the thread synchronisation, and the .release.cluster form costs ~1100 cycles (measured).
 __device__ __forceinline__ void arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -671,7 +674,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     uint64_t* tempty_bar = tfull_bar + 1;                                 // leader: both epilogues drained
     uint64_t* done_bar = tempty_bar + 1;
     uint64_t* boxgo_bar = done_bar + 1;                                   // store slot hand-over (store_boxes)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(boxgo_bar + 2 * kEpi1Warps);
+    uint64_t* edrained_bar = boxgo_bar + 2 * kEpi1Warps;                  // peer: its epilogue drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(edrained_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -685,7 +689,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
         mbar_init(smem_u32(tfull_bar), 1);
-        mbar_init(smem_u32(tempty_bar), 2 * kEpi1Warps);
+        // the leader's epilogue warps arrive on it locally, the peer's drain as one forwarded arrival
+        mbar_init(smem_u32(tempty_bar), kEpi1Warps + 1);
+        mbar_init(smem_u32(edrained_bar), kEpi1Warps);
         mbar_init(smem_u32(done_bar), 1);
         for (int b = 0; b < 2 * kEpi1Warps; ++b) mbar_init(smem_u32(&boxgo_bar[b]), 1);
         *abort_flag = 0u;
@@ -789,16 +795,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             if (elect_one()) mma_commit_local_pair(smem_u32(done_bar));
             __syncwarp();
             mbar_wait_cl(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+        } else {
+            // The peer's MMA warp forwards its CTA's drained accumulator to the leader as one
+            // remote arrival per tile, so the epilogue warps arrive locally (cheap) and one remote
+            // arrival crosses the pair.
+            const uint32_t tempty_leader = map_rank(smem_u32(tempty_bar), 0);
+            int local = 0;
+            for (int t = pair; t < ntiles; t += npairs, ++local) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(edrained_bar), (uint32_t)local & 1u, abort_flag, p.flags,
+                                                       p.budget_ns)))
+                    break;
+                if (lane == 0) arrive_cluster(tempty_leader);
+                __syncwarp();
+            }
         }
     } else if (warp < 2 + kEpi1Warps) {
         // ------------------------------- epilogue (both CTAs) --------------------------------
         // As in the 1-SM kernel: 16 warps x 64 columns of this CTA's 128 accumulator rows, TMEM
-        // released (on the leader's barrier) before the TMA stores.
+        // released before the TMA stores: on the leader's barrier directly (leader CTA) or through
+        // the peer's forwarding warp.
         const int ew = warp - 2;
         const int q = warp & 3;
         const int cq = ew >> 2;
         const float alpha = __fmul_rn(*p.sta, *p.stb);
-        const uint32_t tempty_leader = map_rank(smem_u32(tempty_bar), 0);
+        const uint32_t drained = smem_u32(rank == 0 ? tempty_bar : edrained_bar);
         int local = 0;
         bool ok = true;
         for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
@@ -813,7 +833,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) arrive_cluster(tempty_leader);
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(drained) : "memory");
             ok = store_boxes<k2StoreSlots>(&tmD, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
                                            tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag);
         }
