@@ -57,19 +57,21 @@ __device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */)
 }
 
 // The same decision without computing the threshold, on a = min(|u|, 6) (6 itself encodes 7):
-//   a in [1, 6]:   r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + (0x3FFFFF - 64 r16) carries
-//                  into bit 22, so the code is ((bits(a) + 0x3FFFFF - 64 r16) >> 22) - 252 (the
-//                  code of the lower neighbour is (bits(a) >> 22) - 252);
-//   a in [.5, 1):  likewise with 0x7FFFFF - 128 r16 and a carry into bit 23;
-//   a in [0, .5):  r16 < a * 2^17, compared in fp32 (both sides exact).
+//   a in [1, 6]:  r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + (0x3FFFFF - 64 r16) carries into
+//                 bit 22, so the code is ((bits(a) + 0x3FFFFF - 64 r16) >> 22) - 252 (the code of
+//                 the lower neighbour is (bits(a) >> 22) - 252);
+//   a in [0, 1):  with c = ceil(a * 2^17) (exact: a * 2^17 is one exact product, and adding 2^23
+//                 rounding upward lands on 2^23 + c), the grid is {0, .5, 1} in steps of 2^16 units
+//                 of c, and the code is (c + 65535 - r16) >> 16: below .5 that is 1 iff r16 < c,
+//                 from .5 up it is 1 + [r16 < c - 65536].
 __device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
     const uint32_t b = __float_as_uint(u);
     const float af = fminf(fabsf(u), 6.0f);
     const uint32_t a = __float_as_uint(af);
     const uint32_t hi = (a + (0x3FFFFFu - (252u << 22)) - (r16 << 6)) >> 22;
-    const uint32_t mid = (a + (0x7FFFFFu - (125u << 23)) - (r16 << 7)) >> 23;
-    const uint32_t lo = __uint2float_rn(r16) < __fmul_rn(af, 131072.0f) ? 1u : 0u;
-    const uint32_t code = af >= 1.0f ? hi : (af >= 0.5f ? mid : lo);
+    const uint32_t cb = __float_as_uint(__fadd_ru(__fmul_rn(af, 131072.0f), 8388608.0f));   // 0x4B000000 + c
+    const uint32_t lo = (cb + (65535u - 0x4B000000u) - r16) >> 16;
+    const uint32_t code = a >= 0x3F800000u ? hi : lo;
     return ((b >> 28) & 8u) | code;
 }
 
