@@ -576,14 +576,15 @@ int ora_gemm_full(const uint8_t* a_codes, const uint8_t* a_scales_rm, float a_st
 }
 
 /* ------------------------------------------------------------------------------------ */
-/* GeLU glue of the one-FFN training step (not part of the pages' method): erf form,       */
-/* evaluated in fp64 and rounded to bf16.                                                  */
+/* GeLU glue of the one-FFN training step (not part of the pages' method): exact (erf)     */
+/* form g = x * Phi(x), evaluated in fp64 and rounded to bf16.  Phi(x) = erfc(-x/sqrt 2)/2:  */
+/* the same function as (1 + erf(x/sqrt 2))/2 without its cancellation for negative x.     */
 /* ------------------------------------------------------------------------------------ */
 void ora_gelu_fwd(const uint16_t* h, int64_t n, uint16_t* g)
 {
     for (int64_t i = 0; i < n; ++i) {
         double x = ora_bf16_to_f32(h[i]);
-        double y = 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+        double y = 0.5 * x * erfc(-x / sqrt(2.0));
         g[i] = ora_f32_to_bf16((float)y);
     }
 }
@@ -595,7 +596,7 @@ void ora_gelu_bwd(const uint16_t* h, const uint16_t* dg, int64_t n, uint16_t* dh
     for (int64_t i = 0; i < n; ++i) {
         double x = ora_bf16_to_f32(h[i]);
         double d = ora_bf16_to_f32(dg[i]);
-        double cdf = 0.5 * (1.0 + erf(x / sqrt(2.0)));
+        double cdf = 0.5 * erfc(-x / sqrt(2.0));
         double pdf = inv_sqrt_2pi * exp(-0.5 * x * x);
         dh[i] = ora_f32_to_bf16((float)(d * (cdf + x * pdf)));
     }
