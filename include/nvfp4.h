@@ -185,8 +185,10 @@ nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linea
 nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float* dw,
                               nvfp4_linear_ctx* ctx, nvfp4_stream_t stream);
 
-/* GeLU glue of the one-FFN training step (erf form, fp32 math, bf16 in and out):
- * g = 0.5 h (1 + erf(h / sqrt 2));  dh = dg * (Phi(h) + h phi(h)).  n elements, contiguous. */
+/* GeLU glue of the one-FFN training step (exact erf form, fp32 math, bf16 in and out; the pages
+ * do not describe the activation): g = h Phi(h) with Phi(h) = erfc(-h / sqrt 2) / 2;
+ * dh = dg * (Phi(h) + h phi(h)), phi the N(0,1) density.  n elements, contiguous; results are
+ * within one bf16 step of the exact values rounded to bf16. */
 nvfp4_status nvfp4_gelu_fwd(const void* h, void* g, int64_t n, nvfp4_stream_t stream);
 nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n,
                             nvfp4_stream_t stream);

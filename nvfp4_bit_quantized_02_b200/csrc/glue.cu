@@ -1,7 +1,8 @@
 // glue.cu -- GeLU forward/backward for the one-FFN training step (bf16 in/out, fp32 math).
-// The pages do not describe the activation; the FFN step uses the erf form:
-//   g  = 0.5 h (1 + erf(h / sqrt 2))
-//   dh = dg * (Phi(h) + h * phi(h)),  Phi(h) = 0.5 (1 + erf(h / sqrt 2)),  phi = N(0,1) density.
+// The pages do not describe the activation; the FFN step uses the exact (erf) form:
+//   g  = h Phi(h),  Phi(h) = 0.5 erfc(-h / sqrt 2)  (= 0.5 (1 + erf(h / sqrt 2)) without the
+//        cancellation of 1 + erf for negative h)
+//   dh = dg * (Phi(h) + h * phi(h)),  phi = N(0,1) density.
 // HBM-bound elementwise kernels: 16-byte loads and stores, grid-stride.
 #include <cuda_runtime.h>
 
@@ -12,10 +13,10 @@
 
 namespace nvfp4 {
 
-__device__ __forceinline__ float gelu_f(float h) { return 0.5f * h * (1.0f + erff(h * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_f(float h) { return 0.5f * h * erfcf(h * -0.70710678118654752f); }
 
 __device__ __forceinline__ float gelu_grad_f(float h) {
-    const float cdf = 0.5f * (1.0f + erff(h * 0.70710678118654752f));
+    const float cdf = 0.5f * erfcf(h * -0.70710678118654752f);
     const float pdf = 0.39894228040143268f * expf(-0.5f * h * h);
     return cdf + h * pdf;
 }

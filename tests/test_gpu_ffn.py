@@ -1,0 +1,124 @@
+"""The one-FFN training step (up-projection, GeLU, down-projection; forward and backward) on the
+GPU against the oracle, and the GeLU kernels on their own.
+
+Forward:  H = X W1^T,  G = GeLU(H),  Y = G W2^T.
+Backward: dG = dY W2,  dW2 = dY^T G,  dH = dG * GeLU'(H),  dX = dH W1,  dW1 = dH^T X.
+Every GEMM is an NVFP4 linear of the pages' recipe (gist.science "Pretraining Large Language
+Models with NVFP4", 2.B: 16x16 weights reused transposed, RHT on the wgrad operands, SR on the
+gradients); the GeLU is the glue between them (not in the pages; exact erf form).
+
+Quantization decisions depend on the exact input bits, so the chain is checked link by link:
+each GPU stage is compared with the oracle fed that stage's GPU inputs.  Quantized forms must
+match bit for bit, GEMM outputs stay within |D - D_ref| <= 1e-5 sum|a b| (+ 2^-8 |D_ref| for
+bf16), GeLU outputs within one bf16 step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_helpers import assert_form_equal, bf16_to_f64, check_gemm, nv, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _ulps(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    def line(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)
+    return np.abs(line(a) - line(b))
+
+
+def _gelu_inputs(n: int, seed: int) -> torch.Tensor:
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    parts = [torch.randn(n // 4, generator=g) * s for s in (1e-3, 0.5, 2.0, 6.0)]
+    special = torch.tensor([0.0, -0.0, 1.0, -1.0, -4.0, -6.0, -9.0, -12.0, -20.0, 10.0, 40.0, 1e-30, -1e-30])
+    x = torch.cat(parts + [special])[:n] if n >= special.numel() else special[:n]
+    if x.numel() < n:
+        x = torch.cat([x, torch.randn(n - x.numel(), generator=g)])
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 1000, 65536 + 13])
+def test_gelu_kernels_within_one_bf16_step(n):
+    m = nv()
+    h = _gelu_inputs(n, seed=n)
+    dg = (torch.randn(n, generator=torch.Generator().manual_seed(n + 1)) * 1e-3).to(torch.bfloat16)
+    g = m.nvfp4_gelu_fwd(to_device_bf16(h))
+    dh = m.nvfp4_gelu_bwd(to_device_bf16(h), to_device_bf16(dg))
+    hb, dgb = synth.bf16_bits(h), synth.bf16_bits(dg)
+    for what, got, ref in (("fwd", _bits(g), oracle.gelu_fwd(hb)), ("bwd", _bits(dh), oracle.gelu_bwd(hb, dgb))):
+        d = _ulps(got, ref)
+        assert d.max() <= 1, f"{what}: {int((d > 1).sum())} elements more than one bf16 step off, worst {int(d.max())}"
+        if n >= 1000:
+            assert np.mean(d == 0) > 0.98, what
+
+
+def _check_linear_forms(ctx, xb, wb, rht_seed):
+    xq = oracle.quantize(xb)
+    xq_rht = oracle.quantize(xb, along=1, rht=True, rht_seed=rht_seed)
+    wq = oracle.quantize(wb, block=oracle.BLOCK_16x16)
+    wqt = oracle.transpose_2d(wq)
+    for name, q in (("xq", xq), ("xq_rht", xq_rht), ("wq", wq), ("wqt", wqt)):
+        assert_form_equal(getattr(ctx, name), q, name)
+    return dict(xq=xq, xq_rht=xq_rht, wq=wq, wqt=wqt)
+
+
+def _check_grad_forms(ctx, dyb, rht_seed, sr_seed):
+    dyq = oracle.quantize(dyb, mode=oracle.SR, sr_seed=sr_seed, stream_id=1)
+    dyq_rht = oracle.quantize(dyb, along=1, mode=oracle.SR, rht=True, rht_seed=rht_seed, sr_seed=sr_seed, stream_id=2)
+    assert_form_equal(ctx.dyq, dyq, "dyq")
+    assert_form_equal(ctx.dyq_rht, dyq_rht, "dyq_rht")
+    return dyq, dyq_rht
+
+
+@pytest.mark.parametrize("T,d,f", [(256, 128, 512), (128, 192, 256)])
+def test_ffn_step_chain(T, d, f):
+    m = nv()
+    rht_seed = 0
+    x = synth.activations(T, d, seed=0, outlier_frac=0.01)
+    w1 = synth.weights(f, d, seed=1)
+    w2 = synth.weights(d, f, seed=3)
+    dy = synth.grad_output(T, d, seed=4)
+    up = m.LinearContext(T, d, f, rht_seed=rht_seed)
+    down = m.LinearContext(T, f, d, rht_seed=rht_seed)
+
+    # forward
+    h = m.nvfp4_linear_fwd(up, to_device_bf16(x), to_device_bf16(w1))
+    o_up = _check_linear_forms(up, synth.bf16_bits(x), synth.bf16_bits(w1), rht_seed)
+    ref, s = oracle.gemm_full(o_up["xq"], o_up["wq"])
+    check_gemm(bf16_to_f64(h), ref, s, True, "H = X W1^T")
+
+    g = m.nvfp4_gelu_fwd(h)
+    hb = _bits(h)
+    assert _ulps(_bits(g), oracle.gelu_fwd(hb)).max() <= 1, "G = GeLU(H)"
+
+    y = m.nvfp4_linear_fwd(down, g, to_device_bf16(w2))
+    gb = _bits(g)
+    o_down = _check_linear_forms(down, gb, synth.bf16_bits(w2), rht_seed)
+    ref, s = oracle.gemm_full(o_down["xq"], o_down["wq"])
+    check_gemm(bf16_to_f64(y), ref, s, True, "Y = G W2^T")
+
+    # backward through the down-projection
+    dg, dw2 = m.nvfp4_linear_bwd(down, to_device_bf16(dy), 5)
+    dyq, dyq_rht = _check_grad_forms(down, synth.bf16_bits(dy), rht_seed, 5)
+    ref, s = oracle.gemm_full(dyq, o_down["wqt"])
+    check_gemm(bf16_to_f64(dg), ref, s, True, "dG = dY W2")
+    ref, s = oracle.gemm_full(dyq_rht, o_down["xq_rht"])
+    check_gemm(dw2.cpu().numpy(), ref, s, False, "dW2 = dY^T G")
+
+    dh = m.nvfp4_gelu_bwd(h, dg)
+    assert _ulps(_bits(dh), oracle.gelu_bwd(hb, _bits(dg))).max() <= 1, "dH = dG GeLU'(H)"
+
+    # backward through the up-projection
+    dx, dw1 = m.nvfp4_linear_bwd(up, dh, 6)
+    dhq, dhq_rht = _check_grad_forms(up, _bits(dh), rht_seed, 6)
+    ref, s = oracle.gemm_full(dhq, o_up["wqt"])
+    check_gemm(bf16_to_f64(dx), ref, s, True, "dX = dH W1")
+    ref, s = oracle.gemm_full(dhq_rht, o_up["xq_rht"])
+    check_gemm(dw1.cpu().numpy(), ref, s, False, "dW1 = dH^T X")
+    assert m.nvfp4_poll(up.ws) == 0 and m.nvfp4_poll(down.ws) == 0
