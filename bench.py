@@ -298,6 +298,94 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------------------
+# --workload ffn: the one-FFN training step (up-projection, GeLU, down-projection; forward and
+# backward: six NVFP4 GEMMs, every quantize, both GeLU kernels) at T=16384, 5120 -> 20480 -> 5120
+# ---------------------------------------------------------------------------------------
+FFN_T, FFN_D, FFN_F = 16384, 5120, 20480
+FFN_FLOP = 6 * 2 * FFN_T * FFN_D * FFN_F
+
+
+def run_ffn(args, rank, world, local_rank):
+    import nvfp4_bit_quantized_02_b200 as nv
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = torch.distributed if world > 1 else None
+    x = synth.activations(FFN_T, FFN_D, seed=0, outlier_frac=0.001).to(dev)
+    w1 = synth.weights(FFN_F, FFN_D, seed=1).to(dev)
+    w2 = synth.weights(FFN_D, FFN_F, seed=3).to(dev)
+    dy = synth.grad_output(FFN_T, FFN_D, seed=4).to(dev)
+    up = nv.LinearContext(FFN_T, FFN_D, FFN_F, rht_seed=0, device=dev)
+    down = nv.LinearContext(FFN_T, FFN_F, FFN_D, rht_seed=0, device=dev)
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    h, g, dg, dh = (torch.empty((FFN_T, FFN_F), **bf) for _ in range(4))
+    y, dx = torch.empty((FFN_T, FFN_D), **bf), torch.empty((FFN_T, FFN_D), **bf)
+    dw1 = torch.empty((FFN_F, FFN_D), dtype=torch.float32, device=dev)
+    dw2 = torch.empty((FFN_D, FFN_F), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(seed):
+        nv.nvfp4_linear_fwd(up, x, w1, h)
+        nv.nvfp4_gelu_fwd(h, g)
+        nv.nvfp4_linear_fwd(down, g, w2, y)
+        nv.nvfp4_linear_bwd(down, dy, 2 * seed, dg, dw2)
+        nv.nvfp4_gelu_bwd(h, dg, dh)
+        nv.nvfp4_linear_bwd(up, dh, 2 * seed + 1, dx, dw1)
+
+    # per step: 2 x (W quantize 2 + X/G quantize 2 + fprop 1) + 2 x (dY/dG quantize 2 + dgrad 1
+    # + wgrad 1) + 2 GeLU
+    launches_per_step = 2 * 5 + 2 * 4 + 2
+    for i in range(args.warmup):
+        step(1000 + i)
+    torch.cuda.synchronize()
+    for c in (up, down):
+        if nv.nvfp4_poll(c.ws) != 0:
+            raise RuntimeError("device status after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)                  # evict L2 between steps (outside the events)
+            ev[k][0].record()
+            step(k)
+            ev[k][1].record()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    for c in (up, down):
+        if nv.nvfp4_poll(c.ws) != 0:
+            raise RuntimeError("device status during timing")
+    ms_per_step = reduce_max(sum(a.elapsed_time(b) for a, b in ev), dist, dev) / args.steps
+    if rank != 0:
+        return None
+    return {
+        "metric": "NVFP4 FFN training step TFLOPS at 16384x5120x20480",
+        "value": world * FFN_FLOP / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate; GeLU fp32 math, bf16 in/out",
+        "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W1 and W2, N(0,1e-4) dY; bf16)",
+        "config": {"workload": "one FFN training step: up 5120->20480, GeLU, down 20480->5120, forward and "
+                               "backward (6 GEMMs), weights quantized every step",
+                   "tokens": FFN_T, "d": FFN_D, "ffn": FFN_F, "flop_per_step": FFN_FLOP,
+                   "l2": "256 MiB buffer written between timed steps (outside the events)"},
+        "clocks": clk.summary(),
+        "e2e": None,
+        "gpu_launches": launches_per_step * args.steps,
+        "impl": "ours",
+    }
+
+
+# ---------------------------------------------------------------------------------------
 # the CPU oracle (reference arm and the cpu_baseline field)
 # ---------------------------------------------------------------------------------------
 def cpu_baseline(args, n_cols: int | None = None):
@@ -365,6 +453,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--workload", choices=["linear", "ffn"], default="linear",
+                    help="linear: the 8192x5120x20480 layer (the default line); ffn: the one-FFN step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -385,7 +475,7 @@ def main():
     if rank != 0:
         args.cpu_baseline = False
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_ffn if args.workload == "ffn" else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
