@@ -37,11 +37,11 @@ Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) per GEMM launch, the mean over the fprop, dgrad and wgrad launches
-# of one ncu capture (profiles/gemm_nvf4_kernel_8192x5120x20480.md), valid for the GEMM source
-# it was taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
+# of one ncu capture (profiles/gemm_nvf4_2sm_kernel_8192x5120x20480.md), valid for the GEMM
+# source it was taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
 GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
-GEMM_TRAFFIC = {"sha256": "02ce90f26be9da2f6ebb79bb68d5f60e691abce59a3daf69089311a08e43e634",
-                "bytes_per_launch": 487.7e6}
+GEMM_TRAFFIC = {"sha256": "ee3cbd9f71a8201d5b4146cfc835dcdab133b8dd4f06100c134a4f0a31fc1282",
+                "bytes_per_launch": 486.5e6}
 
 
 def gemm_traffic():
