@@ -129,6 +129,33 @@ nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int6
                                  nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream);
 
 /*
+ * Data-parallel token shards.  The tensor scale comes from the amax of the whole tensor
+ * (gist.science 2.A), so ranks that each hold a shard of the tokens split the two passes and
+ * reduce the amax between them:
+ *   1. nvfp4_amax(shard, rht = 1, rht_seed, ws): the shard's plain amax and the amax after the
+ *      16-point RHT along rows, written as two uint32 fp32 bit patterns at byte offset
+ *      nvfp4_workspace_amax_offset() of ws (reset first).  rows % 16 == 0 when rht = 1.
+ *   2. the caller reduces both words with MAX across ranks (for non-negative floats the bit
+ *      patterns order like the values, so an integer MAX over int32 is exact);
+ *   3. nvfp4_quantize_dual_shard(shard, ..., row_offset, rows_total, ...): pass 2 of
+ *      nvfp4_quantize_dual with the tensor scales of those reduced amaxes.  The shard holds rows
+ *      [row_offset, row_offset + rows) of a rows_total-row tensor, and SR fields are indexed in
+ *      that tensor's forms (row form: (row_offset + r) * cols + c; column form:
+ *      c * rows_total + row_offset + r).
+ * Each shard's forms then equal, bit for bit, its rows (row form) and its K range (column form)
+ * of nvfp4_quantize_dual over the whole tensor.  Shape rules: those of nvfp4_quantize_dual, and
+ * row_offset % 16 == 0, row_offset + rows <= rows_total.  The shard's column form has k = rows.
+ */
+nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, int rht,
+                        uint64_t rht_seed, void* ws, nvfp4_stream_t stream);
+size_t nvfp4_workspace_amax_offset(void);
+nvfp4_status nvfp4_quantize_dual_shard(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                       int64_t row_offset, int64_t rows_total, nvfp4_round mode,
+                                       uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_row,
+                                       uint32_t stream_col, nvfp4_tensor* out_row,
+                                       nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream);
+
+/*
  * 16x16 weight quantization (gist.science 2.B.3), RNE, writing the forward form w_q
  * ([rows][cols], k = cols) and, if w_qt is not NULL, the transposed dgrad form
  * ([cols][rows], k = rows) from the same registers -- bit-identical to nvfp4_transpose_2d of

@@ -8,7 +8,9 @@ no CPU fallback.
 
 The functions carry the C names: ``nvfp4_quantize``, ``nvfp4_quantize_dual``,
 ``nvfp4_quantize_weight``, ``nvfp4_transpose_2d``, ``nvfp4_gemm``, ``nvfp4_linear_fwd``,
-``nvfp4_linear_bwd``, ``nvfp4_gelu_fwd``, ``nvfp4_gelu_bwd``, ``nvfp4_poll``.
+``nvfp4_linear_bwd``, ``nvfp4_gelu_fwd``, ``nvfp4_gelu_bwd``, ``nvfp4_poll``, and for data-parallel
+token shards ``nvfp4_amax``, ``nvfp4_quantize_dual_shard`` (and ``nvfp4_quantize_dual_dp``, which
+all-reduces the amax between them).
 """
 from __future__ import annotations
 
@@ -70,6 +72,9 @@ def _lib():
             "nvfp4_quantize": ([vp, i64, i64, i64, i32, i32, i32, i32, u64, u64, u32, T, vp, vp], i32),
             "nvfp4_quantize_dual": ([vp, i64, i64, i64, i32, u64, u64, u32, u32, T, T, vp, vp], i32),
             "nvfp4_quantize_weight": ([vp, i64, i64, i64, T, T, vp, vp], i32),
+            "nvfp4_amax": ([vp, i64, i64, i64, i32, u64, vp, vp], i32),
+            "nvfp4_workspace_amax_offset": ([], c.c_size_t),
+            "nvfp4_quantize_dual_shard": ([vp, i64, i64, i64, i64, i64, i32, u64, u64, u32, u32, T, T, vp, vp], i32),
             "nvfp4_transpose_2d": ([T, T, vp], i32),
             "nvfp4_gemm": ([T, T, vp, i64, i32, vp, vp], i32),
             "nvfp4_linear_fwd": ([vp, vp, vp, c.POINTER(CLinearCtx), vp], i32),
@@ -122,6 +127,12 @@ class Workspace:
     @property
     def ptr(self):
         return _ptr(self.buf)
+
+    def amax_words(self) -> torch.Tensor:
+        """The two amax words (plain, after the RHT) as an int32 view of the device buffer: fp32
+        bit patterns of non-negative values, so an integer MAX reduction is exact."""
+        off = _lib().nvfp4_workspace_amax_offset()
+        return self.buf[off:off + 8].view(torch.int32)
 
 
 _DEFAULT_WS = {}
@@ -213,6 +224,48 @@ def nvfp4_quantize_dual(x: torch.Tensor, mode: int = RNE, rht_seed: int = 0, sr_
                                     ctypes.byref(a), ctypes.byref(b), ws.ptr, _stream(stream))
     _check(st, "nvfp4_quantize_dual")
     return out_row, out_col
+
+
+def nvfp4_amax(x: torch.Tensor, rht: bool = True, rht_seed: int = 0, ws: Workspace | None = None,
+               stream=None) -> Workspace:
+    """Pass 1 alone: the amax of x (plain, and after the RHT along rows when rht) into ws."""
+    rows, cols, ld = _bf16_2d(x)
+    ws = ws or default_workspace()
+    _check(_lib().nvfp4_amax(_ptr(x), rows, cols, ld, 1 if rht else 0, rht_seed, ws.ptr, _stream(stream)), "nvfp4_amax")
+    return ws
+
+
+def nvfp4_quantize_dual_shard(x: torch.Tensor, row_offset: int, rows_total: int, mode: int = RNE, rht_seed: int = 0,
+                              sr_seed: int = 0, stream_row: int = 0, stream_col: int = 0,
+                              out_row: NVFP4Tensor | None = None, out_col: NVFP4Tensor | None = None,
+                              ws: Workspace | None = None, stream=None):
+    """Pass 2 of nvfp4_quantize_dual for rows [row_offset, row_offset + rows) of a rows_total-row
+    tensor, with the (reduced) amax words already in ws."""
+    rows, cols, ld = _bf16_2d(x)
+    out_row = out_row or NVFP4Tensor.empty(rows, cols, BLOCK_1x16, x.device)
+    out_col = out_col or NVFP4Tensor.empty(cols, rows, BLOCK_1x16, x.device)
+    ws = ws or default_workspace()
+    a, b = out_row.c(), out_col.c()
+    st = _lib().nvfp4_quantize_dual_shard(_ptr(x), rows, cols, ld, row_offset, rows_total, mode, rht_seed, sr_seed,
+                                          stream_row, stream_col, ctypes.byref(a), ctypes.byref(b), ws.ptr,
+                                          _stream(stream))
+    _check(st, "nvfp4_quantize_dual_shard")
+    return out_row, out_col
+
+
+def nvfp4_quantize_dual_dp(x: torch.Tensor, group, row_offset: int, rows_total: int, mode: int = RNE,
+                           rht_seed: int = 0, sr_seed: int = 0, stream_row: int = 0, stream_col: int = 0,
+                           out_row: NVFP4Tensor | None = None, out_col: NVFP4Tensor | None = None,
+                           ws: Workspace | None = None, stream=None):
+    """Both forms of this rank's token shard, equal to the slices of the whole batch's forms: the
+    shard amax, a MAX all-reduce of the two amax words over ``group`` (torch.distributed), then
+    the shard's pass 2."""
+    import torch.distributed as dist
+    ws = nvfp4_amax(x, True, rht_seed, ws, stream)
+    words = ws.amax_words()
+    dist.all_reduce(words, op=dist.ReduceOp.MAX, group=group)
+    return nvfp4_quantize_dual_shard(x, row_offset, rows_total, mode, rht_seed, sr_seed, stream_row, stream_col,
+                                     out_row, out_col, ws, stream)
 
 
 def nvfp4_quantize_weight(w: torch.Tensor, transposed: bool = True, out: NVFP4Tensor | None = None,

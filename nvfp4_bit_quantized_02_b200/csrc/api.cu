@@ -154,6 +154,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
     p.signs = signs;
     p.sr_seed = sr_seed;
     p.flags = &w->flags;
+    p.row_offset = 0;
+    p.rows_total = rows;
     if (along == 0) {
         p.codes_row = out->codes;
         p.scales_row = out->scales;
@@ -177,15 +179,25 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
     return from_cuda(launch_quantize_tiles(p, s));
 }
 
-nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
-                                 uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
-                                 nvfp4_tensor* out_row, nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Both forms of x from one read.  run_amax: pass 1 here (the whole tensor); otherwise the amax
+// words already in ws are used (a token shard whose amax the caller has reduced across ranks).
+// SR fields are indexed in the forms of the rows_total-row tensor of which x is rows
+// [row_offset, row_offset + rows).
+nvfp4_status quantize_dual_impl(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
+                                uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
+                                nvfp4_tensor* out_row, nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream,
+                                int64_t row_offset, int64_t rows_total, bool run_amax) {
     if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
     if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
     if (nvfp4_status st = check_form_buffers(out_row, false)) return st;
     if (nvfp4_status st = check_form_buffers(out_col, false)) return st;
     if (!ws) return NVFP4_ERR_WORKSPACE;
     if (rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (row_offset < 0 || row_offset % 16 != 0 || rows_total < row_offset + rows) return NVFP4_ERR_SHAPE;
     if (nvfp4_status st = check_device()) return st;
     out_row->rows = rows;
     out_row->k = cols;
@@ -200,15 +212,17 @@ nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int6
         return from_cuda(cudaGetLastError());
     }
     Workspace* w = ws_of(ws);
-    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
     if (has_scale_padding(rows, cols))
         if (cudaError_t e = cudaMemsetAsync(out_row->scales, 0, nvfp4_scales_bytes(rows, cols), s)) return from_cuda(e);
     if (has_scale_padding(cols, rows))
         if (cudaError_t e = cudaMemsetAsync(out_col->scales, 0, nvfp4_scales_bytes(cols, rows), s)) return from_cuda(e);
     const uint32_t signs = rht_signs_host(rht_seed);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
-    if (cudaError_t e = launch_amax_rht(xb, rows, cols, ldx, signs, &w->amax_a, &w->amax_b, &w->flags, s))
-        return from_cuda(e);
+    if (run_amax) {
+        if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+        if (cudaError_t e = launch_amax_rht(xb, rows, cols, ldx, signs, &w->amax_a, &w->amax_b, &w->flags, s))
+            return from_cuda(e);
+    }
     QuantParams p;
     std::memset(&p, 0, sizeof(p));
     p.x = xb;
@@ -218,6 +232,8 @@ nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int6
     p.signs = signs;
     p.sr_seed = sr_seed;
     p.flags = &w->flags;
+    p.row_offset = row_offset;
+    p.rows_total = rows_total;
     p.codes_row = out_row->codes;
     p.scales_row = out_row->scales;
     p.st_row = out_row->tensor_scale;
@@ -234,6 +250,43 @@ nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int6
     p.rht_col = 1;
     p.stream_col = stream_col;
     return from_cuda(launch_quantize_tiles(p, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
+                                 uint64_t rht_seed, uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
+                                 nvfp4_tensor* out_row, nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream) {
+    return quantize_dual_impl(x, rows, cols, ldx, mode, rht_seed, sr_seed, stream_row, stream_col, out_row, out_col, ws,
+                              stream, 0, rows, true);
+}
+
+nvfp4_status nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ldx, int rht, uint64_t rht_seed, void* ws,
+                        nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (rht && rows % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Workspace* w = ws_of(ws);
+    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+    if (rows == 0 || cols == 0) return NVFP4_OK;
+    const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+    return from_cuda(rht ? launch_amax_rht(xb, rows, cols, ldx, rht_signs_host(rht_seed), &w->amax_a, &w->amax_b,
+                                           &w->flags, s)
+                         : launch_amax_plain(xb, rows, cols, ldx, &w->amax_a, &w->flags, s));
+}
+
+size_t nvfp4_workspace_amax_offset(void) { return offsetof(Workspace, amax_a); }
+
+nvfp4_status nvfp4_quantize_dual_shard(const void* x, int64_t rows, int64_t cols, int64_t ldx, int64_t row_offset,
+                                       int64_t rows_total, nvfp4_round mode, uint64_t rht_seed, uint64_t sr_seed,
+                                       uint32_t stream_row, uint32_t stream_col, nvfp4_tensor* out_row,
+                                       nvfp4_tensor* out_col, void* ws, nvfp4_stream_t stream) {
+    return quantize_dual_impl(x, rows, cols, ldx, mode, rht_seed, sr_seed, stream_row, stream_col, out_row, out_col, ws,
+                              stream, row_offset, rows_total, false);
 }
 
 nvfp4_status nvfp4_quantize_weight(const void* wp, int64_t rows, int64_t cols, int64_t ldw, nvfp4_tensor* w_q,
@@ -275,6 +328,8 @@ nvfp4_status nvfp4_quantize_weight(const void* wp, int64_t rows, int64_t cols, i
     p.ld = ldw;
     p.block16 = 1;
     p.flags = &w->flags;
+    p.row_offset = 0;
+    p.rows_total = rows;
     p.codes_row = w_q->codes;
     p.scales_row = w_q->scales;
     p.tiles_row = w_q->tile_scales;

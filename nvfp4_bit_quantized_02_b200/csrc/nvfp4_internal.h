@@ -46,6 +46,10 @@ struct QuantParams {
     uint32_t signs;
     uint64_t sr_seed;
     uint32_t* flags;  // workspace flags (timeout of a tile copy)
+    // SR bit indexing of a token shard: x holds rows [row_offset, row_offset + rows) of a
+    // rows_total-row tensor, and SR fields are indexed in the forms of that whole tensor
+    int64_t row_offset;
+    int64_t rows_total;
 };
 
 cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax,

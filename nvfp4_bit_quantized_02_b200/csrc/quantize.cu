@@ -249,7 +249,7 @@ __device__ __forceinline__ uint32_t e4m3_of_amax(float amax_b, float s_enc) {
 template <bool ROW, bool COL>
 __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx, QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31;
     float* s_mult_row = reinterpret_cast<float*>(smem + QuantSmem::mult_row);
     float* s_mult_col = reinterpret_cast<float*>(smem + QuantSmem::mult_col);
     uint8_t* s_tile_code = smem + QuantSmem::tile_code;
@@ -372,7 +372,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t packed = 0;
                 if (sr_row) {
-                    const U4 rw = sr_words(keys, p.stream_row, ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3);
+                    const U4 rw = sr_words(keys, p.stream_row,
+                                           ((uint64_t)(p.row_offset + gr) * (uint64_t)cols + (uint64_t)gc) >> 3);
                     const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -427,9 +428,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
                 }
                 uint32_t c0 = 0, c1 = 0;
                 if (sr_col) {
-                    // form element (column c, row r) has index c * rows + r; the block's first row is a
-                    // multiple of 16, so its 16 fields are Philox calls i0/8 and i0/8 + 1
-                    const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)rows + (uint64_t)(r_base + g * 16)) >> 3;
+                    // form element (column c, row r) has index c * rows_total + row_offset + r; the
+                    // block's first row is a multiple of 16, so its 16 fields are Philox calls i0/8, i0/8 + 1
+                    const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)p.rows_total +
+                                         (uint64_t)(p.row_offset + r_base + g * 16)) >> 3;
                     const U4 w0 = sr_words(keys, p.stream_col, g0);
                     const U4 w1 = sr_words(keys, p.stream_col, g0 + 1);
                     const uint32_t rw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};

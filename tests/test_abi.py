@@ -91,3 +91,17 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(nv, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         nv.lib()
+
+
+def test_shard_entry_points_validate(L):
+    import nvfp4_bit_quantized_02_b200 as nv
+    t = nv.CTensor(16, 16, 0, 16, 0, 0, 0, 0)
+    x, ws = ctypes.c_void_p(16), ctypes.c_void_p(16)
+    assert L.nvfp4_workspace_amax_offset() == 4
+    # amax: no workspace; rows not a multiple of 16 with the RHT
+    assert L.nvfp4_amax(x, 32, 32, 32, 1, 0, None, None) == 5
+    assert L.nvfp4_amax(x, 24, 32, 32, 1, 0, ws, None) == 3
+    # shard: offset not a multiple of 16; shard past the end of the tensor; negative offset
+    assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, 8, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
+    assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, 48, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
+    assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, -16, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
