@@ -11,16 +11,15 @@
 //      magnitude order is the integer order of its low 15 bits), RHT outputs reduced in
 //      fp32; one atomicMax per CTA on the fp32 bit pattern (non-negative floats order like
 //      unsigned ints, and max does not depend on the order of the reduction).
-//   2. quantize: a thread owns a 16-row x 8-column patch (16 x 16-byte loads).  From the same
-//      registers it can emit
+//   2. quantize (quantize_tile_kernel): persistent CTAs take 64 x 256 tiles of x by TMA into
+//      shared memory and emit from one read
 //        - the ROW form (K = columns): a 1x16 block is a lane pair, one shuffle for its amax;
 //          each lane writes 4 code bytes per row (a warp writes 128 contiguous bytes);
-//        - the COL form (K = rows, the transposed wgrad/dgrad operand): a 1x16 block is one
-//          column of the patch, optionally rotated by the 16-point butterfly; codes and
-//          scales are staged in shared memory and written as contiguous row segments.
-//      16x16 tiles (weights) are a lane pair's 16x16 patch; both forms share its scale.
-// The quantize pass walks the tiles in reverse order of the amax pass so its first wave
-// reads what the amax pass left in L2.
+//        - the COL form (K = rows, the transposed wgrad/dgrad operand): a 1x16 block is 16
+//          values down one column of the tile, optionally rotated by the 16-point butterfly;
+//          codes and scales are staged in shared memory and leave as contiguous row segments.
+//      16x16 tiles (weights) share one scale between both forms.  The pass walks the tiles in
+//      reverse order of the amax pass so its first wave reads what the amax pass left in L2.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
