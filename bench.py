@@ -325,17 +325,27 @@ def run_ffn(args, rank, world, local_rank):
     dw2 = torch.empty((FFN_D, FFN_F), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    fused = args.ffn_fused_amax
+
     def step(seed):
         nv.nvfp4_linear_fwd(up, x, w1, h)
-        nv.nvfp4_gelu_fwd(h, g)
+        if fused:   # the GeLU kernels reduce their output's amax; G's and dH's quantize skip pass 1
+            nv.nvfp4_gelu_fwd_amax(h, g, rht_seed=0, ws=down.ws)
+            down.amax_ready = True
+        else:
+            nv.nvfp4_gelu_fwd(h, g)
         nv.nvfp4_linear_fwd(down, g, w2, y)
         nv.nvfp4_linear_bwd(down, dy, 2 * seed, dg, dw2)
-        nv.nvfp4_gelu_bwd(h, dg, dh)
+        if fused:
+            nv.nvfp4_gelu_bwd_amax(h, dg, dh, rht_seed=0, ws=up.ws)
+            up.amax_ready = True
+        else:
+            nv.nvfp4_gelu_bwd(h, dg, dh)
         nv.nvfp4_linear_bwd(up, dh, 2 * seed + 1, dx, dw1)
 
-    # per step: 2 x (W quantize 2 + X/G quantize 2 + fprop 1) + 2 x (dY/dG quantize 2 + dgrad 1
-    # + wgrad 1) + 2 GeLU
-    launches_per_step = 2 * 5 + 2 * 4 + 2
+    # per step: 2 x (W quantize 2 + X/G quantize 2 + fprop 1) + 2 x (dY/dH quantize 2 + dgrad 1
+    # + wgrad 1) + 2 GeLU; the fused variant drops the amax passes of G and dH
+    launches_per_step = 2 * 5 + 2 * 4 + 2 - (2 if fused else 0)
     for i in range(args.warmup):
         step(1000 + i)
     torch.cuda.synchronize()
@@ -375,7 +385,8 @@ def run_ffn(args, rank, world, local_rank):
         "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate; GeLU fp32 math, bf16 in/out",
         "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W1 and W2, N(0,1e-4) dY; bf16)",
         "config": {"workload": "one FFN training step: up 5120->20480, GeLU, down 20480->5120, forward and "
-                               "backward (6 GEMMs), weights quantized every step",
+                               "backward (6 GEMMs), weights quantized every step"
+                               + (", amax of G and dH fused into the GeLU kernels" if fused else ""),
                    "tokens": FFN_T, "d": FFN_D, "ffn": FFN_F, "flop_per_step": FFN_FLOP,
                    "l2": "256 MiB buffer written between timed steps (outside the events)"},
         "clocks": clk.summary(),
@@ -455,6 +466,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--workload", choices=["linear", "ffn"], default="linear",
                     help="linear: the 8192x5120x20480 layer (the default line); ffn: the one-FFN step")
+    ap.add_argument("--ffn-fused-amax", action="store_true",
+                    help="ffn: the GeLU kernels that also reduce their output's amax (slower as they stand)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

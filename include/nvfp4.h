@@ -199,10 +199,14 @@ typedef struct {
     nvfp4_tensor xq, xq_rht, wq, wqt, dyq, dyq_rht;
     void* ws;
     int32_t w_cached;
-    int32_t reserved;
+    /* nonzero: the amax words of the next call's input (x for nvfp4_linear_fwd, dy for
+     * nvfp4_linear_bwd) are already in ws, written by a producer that fused them
+     * (nvfp4_gelu_fwd_amax, nvfp4_gelu_bwd_amax, or nvfp4_amax + a reduction); the call then
+     * skips its amax pass and sets the field back to 0 */
+    int32_t amax_ready;
 } nvfp4_linear_ctx;
 
-/* Forward: quantize W (16x16, both layouts) unless cached, quantize X (both forms), then
+/* Forward: quantize X (both forms), quantize W (16x16, both layouts) unless cached, then
  * y[T][n] (bf16) = GEMM(xq, wq). */
 nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linear_ctx* ctx,
                               nvfp4_stream_t stream);
@@ -219,6 +223,16 @@ nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float*
 nvfp4_status nvfp4_gelu_fwd(const void* h, void* g, int64_t n, nvfp4_stream_t stream);
 nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n,
                             nvfp4_stream_t stream);
+
+/* The GeLU kernels with the amax of their bf16 output fused in: out[rows][cols] (contiguous) as
+ * above, and in ws (reset first) the plain amax and the amax after the 16-point RHT (rht_seed)
+ * along rows of out, as nvfp4_amax would compute them from out.  Set the consuming linear
+ * context's amax_ready (same ws, same rht_seed) to skip that layer's amax pass.  Shape rules:
+ * rows % 16 == 0, cols % 16 == 0. */
+nvfp4_status nvfp4_gelu_fwd_amax(const void* h, void* g, int64_t rows, int64_t cols, uint64_t rht_seed,
+                                 void* ws, nvfp4_stream_t stream);
+nvfp4_status nvfp4_gelu_bwd_amax(const void* h, const void* dg, void* dh, int64_t rows, int64_t cols,
+                                 uint64_t rht_seed, void* ws, nvfp4_stream_t stream);
 
 /*
  * nvfp4_quantize without a workspace argument.  The pages have no counterpart: this exists for

@@ -48,7 +48,7 @@ class CLinearCtx(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("n", ctypes.c_int64), ("rht_seed", ctypes.c_uint64),
                 ("xq", CTensor), ("xq_rht", CTensor), ("wq", CTensor), ("wqt", CTensor), ("dyq", CTensor),
                 ("dyq_rht", CTensor), ("ws", ctypes.c_void_p), ("w_cached", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("amax_ready", ctypes.c_int32)]
 
 
 _L = None
@@ -81,6 +81,8 @@ def _lib():
             "nvfp4_linear_bwd": ([vp, u64, vp, vp, c.POINTER(CLinearCtx), vp], i32),
             "nvfp4_gelu_fwd": ([vp, vp, i64, vp], i32),
             "nvfp4_gelu_bwd": ([vp, vp, vp, i64, vp], i32),
+            "nvfp4_gelu_fwd_amax": ([vp, vp, i64, i64, u64, vp, vp], i32),
+            "nvfp4_gelu_bwd_amax": ([vp, vp, vp, i64, i64, u64, vp, vp], i32),
             "nvfp4_poll": ([vp, vp], i32),
             "nvfp4_set_wait_budget_ns": ([u64], None),
             "nvfp4_status_string": ([i32], c.c_char_p),
@@ -318,6 +320,32 @@ def nvfp4_gelu_bwd(h: torch.Tensor, dg: torch.Tensor, out: torch.Tensor | None =
     return out
 
 
+def nvfp4_gelu_fwd_amax(h: torch.Tensor, out: torch.Tensor | None = None, rht_seed: int = 0,
+                        ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """GeLU of h [rows][cols] with the plain and RHT amax of the bf16 result into ws."""
+    rows, cols, ld = _bf16_2d(h)
+    if ld != cols:
+        raise ValueError("nvfp4_gelu_fwd_amax needs a contiguous input")
+    out = torch.empty_like(h) if out is None else out
+    ws = ws or default_workspace()
+    _check(_lib().nvfp4_gelu_fwd_amax(_ptr(h), _ptr(out), rows, cols, rht_seed, ws.ptr, _stream(stream)),
+           "nvfp4_gelu_fwd_amax")
+    return out
+
+
+def nvfp4_gelu_bwd_amax(h: torch.Tensor, dg: torch.Tensor, out: torch.Tensor | None = None, rht_seed: int = 0,
+                        ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """dg * GeLU'(h) with the plain and RHT amax of the bf16 result into ws."""
+    rows, cols, ld = _bf16_2d(h)
+    if ld != cols or not dg.is_contiguous():
+        raise ValueError("nvfp4_gelu_bwd_amax needs contiguous inputs")
+    out = torch.empty_like(h) if out is None else out
+    ws = ws or default_workspace()
+    _check(_lib().nvfp4_gelu_bwd_amax(_ptr(h), _ptr(dg), _ptr(out), rows, cols, rht_seed, ws.ptr, _stream(stream)),
+           "nvfp4_gelu_bwd_amax")
+    return out
+
+
 # ---------------------------------------------------------------------------------------
 # linear layer
 # ---------------------------------------------------------------------------------------
@@ -344,6 +372,16 @@ class LinearContext:
     @w_cached.setter
     def w_cached(self, v: bool):
         self.ctx.w_cached = 1 if v else 0
+
+    @property
+    def amax_ready(self) -> bool:
+        """The next call's input has its amax words in this context's workspace already (a fused
+        producer wrote them); the call skips its amax pass and clears the flag."""
+        return bool(self.ctx.amax_ready)
+
+    @amax_ready.setter
+    def amax_ready(self, v: bool):
+        self.ctx.amax_ready = 1 if v else 0
 
 
 def nvfp4_linear_fwd(ctx: LinearContext, x: torch.Tensor, w: torch.Tensor | None, y: torch.Tensor | None = None,

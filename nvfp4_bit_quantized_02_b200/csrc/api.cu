@@ -400,14 +400,16 @@ static nvfp4_status check_ctx(const nvfp4_linear_ctx* c) {
 nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linear_ctx* ctx, nvfp4_stream_t stream) {
     if (nvfp4_status st = check_ctx(ctx)) return st;
     if (!x || !y || (!w && !ctx->w_cached)) return NVFP4_ERR_NULL;
-    nvfp4_status st;
+    // X first: with amax_ready its amax words are in ws, which the weight's quantize overwrites
+    const bool ready = ctx->amax_ready != 0;
+    ctx->amax_ready = 0;
+    nvfp4_status st = quantize_dual_impl(x, ctx->T, ctx->d, ctx->d, NVFP4_RNE, ctx->rht_seed, 0, 0, 0, &ctx->xq,
+                                         &ctx->xq_rht, ctx->ws, stream, 0, ctx->T, !ready);
+    if (st) return st;
     if (!ctx->w_cached) {
         st = nvfp4_quantize_weight(w, ctx->n, ctx->d, ctx->d, &ctx->wq, &ctx->wqt, ctx->ws, stream);
         if (st) return st;
     }
-    st = nvfp4_quantize_dual(x, ctx->T, ctx->d, ctx->d, NVFP4_RNE, ctx->rht_seed, 0, 0, 0, &ctx->xq, &ctx->xq_rht, ctx->ws,
-                             stream);
-    if (st) return st;
     return nvfp4_gemm(&ctx->xq, &ctx->wq, y, ctx->n, NVFP4_OUT_BF16, ctx->ws, stream);
 }
 
@@ -415,8 +417,10 @@ nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float*
                               nvfp4_stream_t stream) {
     if (nvfp4_status st = check_ctx(ctx)) return st;
     if (!dy) return NVFP4_ERR_NULL;
-    nvfp4_status st = nvfp4_quantize_dual(dy, ctx->T, ctx->n, ctx->n, NVFP4_SR, ctx->rht_seed, sr_seed, NVFP4_STREAM_DGRAD,
-                                          NVFP4_STREAM_WGRAD, &ctx->dyq, &ctx->dyq_rht, ctx->ws, stream);
+    const bool ready = ctx->amax_ready != 0;
+    ctx->amax_ready = 0;
+    nvfp4_status st = quantize_dual_impl(dy, ctx->T, ctx->n, ctx->n, NVFP4_SR, ctx->rht_seed, sr_seed, NVFP4_STREAM_DGRAD,
+                                         NVFP4_STREAM_WGRAD, &ctx->dyq, &ctx->dyq_rht, ctx->ws, stream, 0, ctx->T, !ready);
     if (st) return st;
     if (dx) {
         st = nvfp4_gemm(&ctx->dyq, &ctx->wqt, dx, ctx->d, NVFP4_OUT_BF16, ctx->ws, stream);
@@ -447,6 +451,33 @@ nvfp4_status nvfp4_gelu_bwd(const void* h, const void* dg, void* dh, int64_t n, 
     if (nvfp4_status st = check_device()) return st;
     return from_cuda(launch_gelu_bwd(reinterpret_cast<const uint16_t*>(h), reinterpret_cast<const uint16_t*>(dg),
                                      reinterpret_cast<uint16_t*>(dh), n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static nvfp4_status gelu_amax(bool bwd, const void* h, const void* dg, void* out, int64_t rows, int64_t cols,
+                              uint64_t rht_seed, void* ws, nvfp4_stream_t stream) {
+    if (rows < 0 || cols < 0 || rows % 16 != 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (rows > 0 && cols > 0) {
+        if (!h || !out || (bwd && !dg)) return NVFP4_ERR_NULL;
+        if (!aligned16(h) || !aligned16(out) || (bwd && !aligned16(dg))) return NVFP4_ERR_ALIGN;
+    }
+    if (nvfp4_status st = check_device()) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaError_t e = reset_amax(ws, s)) return from_cuda(e);
+    Workspace* w = ws_of(ws);
+    return from_cuda(launch_gelu_amax(bwd, reinterpret_cast<const uint16_t*>(h), reinterpret_cast<const uint16_t*>(dg),
+                                      reinterpret_cast<uint16_t*>(out), rows, cols, rht_signs_host(rht_seed), &w->amax_a,
+                                      &w->amax_b, &w->flags, s));
+}
+
+nvfp4_status nvfp4_gelu_fwd_amax(const void* h, void* g, int64_t rows, int64_t cols, uint64_t rht_seed, void* ws,
+                                 nvfp4_stream_t stream) {
+    return gelu_amax(false, h, nullptr, g, rows, cols, rht_seed, ws, stream);
+}
+
+nvfp4_status nvfp4_gelu_bwd_amax(const void* h, const void* dg, void* dh, int64_t rows, int64_t cols, uint64_t rht_seed,
+                                 void* ws, nvfp4_stream_t stream) {
+    return gelu_amax(true, h, dg, dh, rows, cols, rht_seed, ws, stream);
 }
 
 nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream) {

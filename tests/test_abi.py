@@ -105,3 +105,11 @@ def test_shard_entry_points_validate(L):
     assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, 8, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
     assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, 48, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
     assert L.nvfp4_quantize_dual_shard(x, 32, 32, 32, -16, 64, 0, 0, 0, 1, 2, ctypes.byref(t), ctypes.byref(t), ws, None) == 3
+
+
+def test_gelu_amax_entry_points_validate(L):
+    h, ws = ctypes.c_void_p(16), ctypes.c_void_p(16)
+    assert L.nvfp4_gelu_fwd_amax(h, h, 32, 32, 0, None, None) == 5       # no workspace
+    assert L.nvfp4_gelu_fwd_amax(h, h, 24, 32, 0, ws, None) == 3         # rows % 16
+    assert L.nvfp4_gelu_bwd_amax(h, None, h, 32, 32, 0, ws, None) == 1    # no dg
+    assert L.nvfp4_gelu_bwd_amax(h, h, ctypes.c_void_p(18), 32, 32, 0, ws, None) == 2   # misaligned output

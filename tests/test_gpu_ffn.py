@@ -58,6 +58,31 @@ def test_gelu_kernels_within_one_bf16_step(n):
             assert np.mean(d == 0) > 0.98, what
 
 
+@pytest.mark.parametrize("rows,cols", [(64, 256), (160, 512)])
+def test_gelu_amax_kernels(rows, cols):
+    # the fused kernels' outputs stay within one bf16 step of the oracle, and the amax words they
+    # leave in the workspace are exactly the oracle's amax of those outputs (plain and after the
+    # RHT along rows)
+    m = nv()
+    g_ = torch.Generator().manual_seed(rows + cols)
+    h = (torch.randn(rows, cols, generator=g_) * 2.0).to(torch.bfloat16)
+    dg = (torch.randn(rows, cols, generator=g_) * 1e-3).to(torch.bfloat16)
+    hb = synth.bf16_bits(h)
+    for bwd in (False, True):
+        ws = m.Workspace()
+        if bwd:
+            out = m.nvfp4_gelu_bwd_amax(to_device_bf16(h), to_device_bf16(dg), rht_seed=7, ws=ws)
+            ref = oracle.gelu_bwd(hb, synth.bf16_bits(dg))
+        else:
+            out = m.nvfp4_gelu_fwd_amax(to_device_bf16(h), rht_seed=7, ws=ws)
+            ref = oracle.gelu_fwd(hb)
+        ob = _bits(out).reshape(rows, cols)
+        assert _ulps(ob.reshape(-1), np.asarray(ref).reshape(-1)).max() <= 1
+        words = ws.amax_words().cpu().numpy().view(np.float32)
+        assert words[0] == np.float32(oracle.quantize(ob).amax), "plain amax"
+        assert words[1] == np.float32(oracle.quantize(ob, along=1, rht=True, rht_seed=7).amax), "RHT amax"
+
+
 def _check_linear_forms(ctx, xb, wb, rht_seed):
     xq = oracle.quantize(xb)
     xq_rht = oracle.quantize(xb, along=1, rht=True, rht_seed=rht_seed)
@@ -76,8 +101,9 @@ def _check_grad_forms(ctx, dyb, rht_seed, sr_seed):
     return dyq, dyq_rht
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("T,d,f", [(256, 128, 512), (128, 192, 256)])
-def test_ffn_step_chain(T, d, f):
+def test_ffn_step_chain(T, d, f, fused):
     m = nv()
     rht_seed = 0
     x = synth.activations(T, d, seed=0, outlier_frac=0.01)
@@ -93,7 +119,11 @@ def test_ffn_step_chain(T, d, f):
     ref, s = oracle.gemm_full(o_up["xq"], o_up["wq"])
     check_gemm(bf16_to_f64(h), ref, s, True, "H = X W1^T")
 
-    g = m.nvfp4_gelu_fwd(h)
+    if fused:   # the GeLU reduces G's amax; the down-projection skips its amax pass
+        g = m.nvfp4_gelu_fwd_amax(h, rht_seed=rht_seed, ws=down.ws)
+        down.amax_ready = True
+    else:
+        g = m.nvfp4_gelu_fwd(h)
     hb = _bits(h)
     assert _ulps(_bits(g), oracle.gelu_fwd(hb)).max() <= 1, "G = GeLU(H)"
 
@@ -111,7 +141,11 @@ def test_ffn_step_chain(T, d, f):
     ref, s = oracle.gemm_full(dyq_rht, o_down["xq_rht"])
     check_gemm(dw2.cpu().numpy(), ref, s, False, "dW2 = dY^T G")
 
-    dh = m.nvfp4_gelu_bwd(h, dg)
+    if fused:
+        dh = m.nvfp4_gelu_bwd_amax(h, dg, rht_seed=rht_seed, ws=up.ws)
+        up.amax_ready = True
+    else:
+        dh = m.nvfp4_gelu_bwd(h, dg)
     assert _ulps(_bits(dh), oracle.gelu_bwd(hb, _bits(dg))).max() <= 1, "dH = dG GeLU'(H)"
 
     # backward through the up-projection
@@ -122,3 +156,4 @@ def test_ffn_step_chain(T, d, f):
     ref, s = oracle.gemm_full(dhq_rht, o_up["xq_rht"])
     check_gemm(dw1.cpu().numpy(), ref, s, False, "dW1 = dH^T X")
     assert m.nvfp4_poll(up.ws) == 0 and m.nvfp4_poll(down.ws) == 0
+    assert not up.amax_ready and not down.amax_ready
