@@ -121,6 +121,15 @@ class ClockSampler:
                 "samples": len(rows), "samples_under_load": len(loaded), "sm_mhz_min": min(sm)}
 
 
+def linear_config() -> dict:
+    """The workload of the default line (both arms report it)."""
+    return {"workload": "NVFP4 linear fwd+bwd: fprop 8192x20480x5120, dgrad 8192x5120x20480, "
+                        "wgrad 20480x5120x8192, W 16x16 quantized every step",
+            "tokens": T_TOK, "d_in": D_IN, "d_out": D_OUT, "rht": "16-point, wgrad operands",
+            "sr": "Philox4x32-10, dY both forms",
+            "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"}
+
+
 # ---------------------------------------------------------------------------------------
 # cross-rank aggregation (weak scaling: every rank runs the whole layer on its own batch)
 # ---------------------------------------------------------------------------------------
@@ -270,11 +279,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W, N(0,1e-4) dY; bf16)",
-        "config": {"workload": "NVFP4 linear fwd+bwd: fprop 8192x20480x5120, dgrad 8192x5120x20480, "
-                               "wgrad 20480x5120x8192, W 16x16 quantized every step",
-                   "tokens": T_TOK, "d_in": D_IN, "d_out": D_OUT, "rht": "16-point, wgrad operands",
-                   "sr": "Philox4x32-10, dY both forms",
-                   "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"},
+        "config": linear_config(),
         "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_2sm_kernel", "achieved": achieved,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
                      "traffic": gemm_traffic(),
@@ -449,7 +454,7 @@ def run_reference(args, rank, world):
     return {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp64 GEMM over dequantized NVFP4 operands (CPU)", "data": "synthetic",
-            "config": {"workload": "NVFP4 linear fwd+bwd, bounded slice of T=8192 d=5120 n=20480 (see cpu_baseline)"},
+            "config": linear_config(),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": samples[0]["cores"], "kind": "oracle",
                              "sample": samples[0]["sample"]},
