@@ -20,18 +20,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // sm_100 check, cached per device
 nvfp4_status check_device() {
-    static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+    static std::atomic<int> cached[64];  // 0 unknown, 1 ok, 2 unsupported (any thread may fill it)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (dev < 0 || dev >= 64) return NVFP4_ERR_UNSUPPORTED;
-    if (cached[dev] == 0) {
+    int c = cached[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-        cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        c = (major == 10 && minor == 0) ? 1 : 2;
+        cached[dev].store(c, std::memory_order_relaxed);
     }
-    return cached[dev] == 1 ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED;
+    return c == 1 ? NVFP4_OK : NVFP4_ERR_UNSUPPORTED;
 }
 
 nvfp4_status from_cuda(cudaError_t e) {

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -908,16 +909,24 @@ static bool make_out_map(CUtensorMap* map, void* d, int64_t M, int64_t N, int64_
     return r == CUDA_SUCCESS;
 }
 
+// The dynamic shared-memory limit is a per-device attribute of a kernel: raise it once on each
+// device (bit d of `done`) before the first launch there.
+static cudaError_t ensure_smem_attr(const void* kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
 cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
                              const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                              void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
                              cudaStream_t stream) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_1sm{0};
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_kernel), kGemmSmem, attr_1sm)) return e;
     CUtensorMap ta, tb;
     if (!make_code_map(&ta, a_codes, M, K, kBM) || !make_code_map(&tb, b_codes, N, K, kBN))
         return cudaErrorInvalidValue;
@@ -949,12 +958,9 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
     const char* variant = getenv("NVFP4_GEMM_VARIANT");
     const bool force_1sm = variant && strcmp(variant, "1sm") == 0;
     if (!force_1sm && M >= 256 && sms >= 2) {
-        static bool attr2_set = false;
-        if (!attr2_set) {
-            cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
-            if (e != cudaSuccess) return e;
-            attr2_set = true;
-        }
+        static std::atomic<uint64_t> attr_2sm{0};
+        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_2sm_kernel), k2Smem, attr_2sm))
+            return e;
         CUtensorMap ta2, tb2;
         if (!make_code_map(&ta2, a_codes, M, K, 128) || !make_code_map(&tb2, b_codes, N, K, 128)) return cudaErrorInvalidValue;
         p.tiles_m = (int32_t)((M + 255) / 256);
