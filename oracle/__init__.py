@@ -9,13 +9,17 @@ Parity status of each function (pins live in ``tests/test_oracle_*.py``):
 - E2M1 / E4M3 encode and decode: pinned against ``ml_dtypes`` (exhaustive on the decision
   ranges) and hand-worked values under ``tests/golden``.
 - Philox4x32-10: pinned on CPU only statistically; pinned exactly on the GPU against cuRAND's
-  independent Philox4_32_10 generator (``tests/test_gpu_philox_curand.py``).
+  independent Philox4_32_10 generator (``tests/test_gpu_encoders.py``).
 - RHT butterfly: pinned against the closed-form Sylvester matrix in fp64, orthogonality and
   the exact one-hot response.
 - SR: pinned by unbiasedness and frequency statistics at 3 sigma over 1e6 draws.
 - Quantizers: pinned by the 6.25 % invariant, the reconstruction bound, the transpose identity
   of 16x16 blocks and a hand-worked block.
 - GEMM: pinned against numpy matmul of operands decoded through ``ml_dtypes``.
+- GeLU glue: pinned against scipy's normal CDF, closed forms and finite differences.
+- MXFP4 quantizer (the pages' comparison format): pinned against an encoder built from
+  ``ml_dtypes`` (E2M1 and E8M0) and numpy's frexp, the scale's closed form per binade and
+  the reconstruction bound (``tests/test_oracle_mx.py``).
 """
 from __future__ import annotations
 
@@ -79,6 +83,10 @@ def lib():
         L.ora_sr_bits16_batch.restype = None
         L.ora_philox_batch.argtypes = [c.c_uint64, c.c_uint32, c.c_uint64, c.c_int64, u32p]
         L.ora_philox_batch.restype = None
+        L.ora_ue8m0_of_amax.argtypes = [c.c_float]
+        L.ora_ue8m0_of_amax.restype = c.c_uint8
+        L.ora_quantize_mx.argtypes = [u16p, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_uint64, c.c_uint32, u8p, u8p]
+        L.ora_quantize_mx.restype = c.c_int
         _LIB = L
     return _LIB
 
@@ -288,3 +296,25 @@ def gelu_bwd(h_bits: np.ndarray, dg_bits: np.ndarray) -> np.ndarray:
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------------------
+# MXFP4 (the pages' comparison format): blocks of 32, UE8M0 scales, no tensor scale
+# ---------------------------------------------------------------------------------------
+def ue8m0_of_amax(amax: float) -> int:
+    """The UE8M0 code of a block with this amax: floor(log2 amax) - 2 + 127, in [0, 254]."""
+    return int(lib().ora_ue8m0_of_amax(float(amax)))
+
+
+def quantize_mx(x_bits: np.ndarray, mode: int = RNE, sr_seed: int = 0, stream_id: int = 0):
+    """MXFP4 of a bf16 tensor [rows][cols] (uint16 bit patterns): codes [rows][cols/2] (even k in
+    the low nibble) and UE8M0 scales [rows][cols/32]."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    st = lib().ora_quantize_mx(_p(x, ctypes.c_uint16), rows, cols, cols, mode, sr_seed, stream_id,
+                               _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8))
+    if st != 0:
+        raise ValueError(f"ora_quantize_mx: status {st}")
+    return codes, scales

@@ -640,3 +640,57 @@ void ora_philox_batch(uint64_t seed, uint32_t stream_id, uint64_t g0, int64_t n,
         ora_philox4x32_10(ctr, key, out4 + 4 * t);
     }
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* MXFP4, the pages' comparison format (gist.science 2.A: blocks of 32 elements, UE8M0    */
+/* scale factors, no tensor scale).  The pages give no rule for the scale; the reading    */
+/* taken is the microscaling one: the block's shared exponent is floor(log2 amax_b) - 2   */
+/* (2 = the largest E2M1 exponent, 6 = 1.5 * 2^2), stored as the UE8M0 code E + 127,      */
+/* clamped to [0, 254] (255 is NaN); an all-zero block gets code 0.  Elements are         */
+/* u = v / 2^E (exact: a power of two), encoded to E2M1 by RNE or SR exactly as NVFP4's,   */
+/* saturating to 6.  SR fields are indexed by the element's row-major position.           */
+/* ------------------------------------------------------------------------------------ */
+uint8_t ora_ue8m0_of_amax(float amax)
+{
+    if (!(amax > 0.0f)) return 0;
+    int e2;
+    (void)frexpf(amax, &e2);          /* amax = m * 2^e2, m in [0.5, 1): floor(log2 amax) = e2 - 1 */
+    int code = (e2 - 1) - 2 + 127;
+    if (code < 0) code = 0;
+    if (code > 254) code = 254;
+    return (uint8_t)code;
+}
+
+/* x [rows][cols] bf16 (leading dimension ld), cols % 32 == 0 -> codes [rows][cols/2] (even k in
+   the low nibble), scales [rows][cols/32] UE8M0. */
+int ora_quantize_mx(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int mode, uint64_t sr_seed,
+                    uint32_t stream_id, uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols) return ORA_ERR_SHAPE;
+    if (mode != 0 && mode != 1) return ORA_ERR_ARG;
+    const int64_t nb = cols / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int t = 0; t < 32; ++t) {
+                float v = ora_bf16_to_f32(x[r * ld + b * 32 + t]);
+                if (isnan(v) || isinf(v)) return ORA_ERR_NONFINITE;
+                amax = fmaxf(amax, fabsf(v));
+            }
+            const uint8_t sc = ora_ue8m0_of_amax(amax);
+            scales[r * nb + b] = sc;
+            const int e = (int)sc - 127;
+            for (int t = 0; t < 32; t += 2) {
+                uint8_t q[2];
+                for (int j = 0; j < 2; ++j) {
+                    const int64_t k = b * 32 + t + j;
+                    const float u = ldexpf(ora_bf16_to_f32(x[r * ld + k]), -e);
+                    q[j] = mode == 0 ? ora_e2m1_rne(u)
+                                     : ora_e2m1_sr(u, ora_sr_bits16(sr_seed, stream_id, (uint64_t)(r * cols + k)));
+                }
+                codes[r * (cols / 2) + (b * 32 + t) / 2] = (uint8_t)(q[0] | (q[1] << 4));
+            }
+        }
+    }
+    return ORA_OK;
+}
