@@ -40,7 +40,7 @@ FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200
 # of one ncu capture (profiles/gemm_nvf4_2sm_kernel_8192x5120x20480.md), valid for the GEMM
 # source it was taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
 GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
-GEMM_TRAFFIC = {"sha256": "9e1fe7a808c02d8869e319e4d300ad9c26cebe96cf16e9024fe76ed384d761b8",
+GEMM_TRAFFIC = {"sha256": "1b1ff1cb88ee135cae6fadffa2b5882b18ff9143af5e688ab53806a543826b35",
                 "bytes_per_launch": 486.5e6}
 
 

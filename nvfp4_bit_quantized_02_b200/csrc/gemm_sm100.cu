@@ -557,7 +557,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 // complete on the leader's full barrier.  The leader CTA (rank 0) then moves the scales into
 // TMEM with tcgen05.cp.cta_group::2 (each CTA from its own shared memory; in a cta_group::2
 // kernel tcgen05.st from scale warps waits for the pair's queued MMAs, ~1400 cycles a stage)
-// and issues the MMAs; commits multicast to both CTAs.  No TMA load uses multicast.
+// and issues the MMAs; its commits arrive in both CTAs.  Every copy is issued by the CTA that
+// owns its destination.
 // ---------------------------------------------------------------------------------------
 constexpr int k2Stages = 5;
 constexpr int k2ABytes = 128 * kBK / 2;                // 16384: this CTA's 128 A rows
