@@ -415,7 +415,7 @@ def cpu_baseline(args, n_cols: int | None = None):
 
     cores = os.cpu_count() or 1
     T_s = 256
-    n_s = n_cols or min(D_OUT, 1024 * max(1, cores // 8))
+    n_s = n_cols or min(D_OUT, 4096 * max(1, cores // 8))   # about 10 s of oracle work
     x = synth.bf16_bits(synth.activations(T_TOK, D_IN, seed=0, outlier_frac=0.001)[:T_s])
     w = synth.bf16_bits(synth.weights(D_OUT, D_IN, seed=1)[:n_s])
     dy = synth.bf16_bits(synth.grad_output(T_TOK, D_OUT, seed=2)[:T_s, :n_s])
