@@ -177,7 +177,9 @@ nvfp4_status nvfp4_transpose_2d(const nvfp4_tensor* w, nvfp4_tensor* wt, nvfp4_s
  * the same k (brainai.pro "Details techniques": the FP4 GEMMs of the fully connected layers).
  * M = a->rows, N = b->rows, K = a->k.  fp32 accumulation in tensor memory; bf16 or fp32 output
  * with leading dimension ldd (elements).  Shape rules: K % 32 == 0 and K > 0; M, N >= 1;
- * ldd >= N and ldd * sizeof(out) % 16 == 0.  ws receives the timeout flag.
+ * ldd >= N and ldd * sizeof(out) % 16 == 0.  ws receives the timeout flag.  For M >= 256 the
+ * call runs the SM-pair kernel (a cluster of two CTAs per 256 x 256 output tile); the environment
+ * variable NVFP4_GEMM_VARIANT=1sm, read on every call, selects the 1-SM kernel for every shape.
  */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, int64_t ldd,
                         nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream);
