@@ -113,3 +113,16 @@ def test_gelu_amax_entry_points_validate(L):
     assert L.nvfp4_gelu_fwd_amax(h, h, 24, 32, 0, ws, None) == 3         # rows % 16
     assert L.nvfp4_gelu_bwd_amax(h, None, h, 32, 32, 0, ws, None) == 1    # no dg
     assert L.nvfp4_gelu_bwd_amax(h, h, ctypes.c_void_p(18), 32, 32, 0, ws, None) == 2   # misaligned output
+
+
+def test_gemm_size_limits_and_degenerate_shapes(L):
+    # sizes past the GEMM's 2^30 limit per dimension are refused before any device work; so are
+    # empty GEMMs (M or N of 0, K of 0)
+    import nvfp4_bit_quantized_02_b200 as nv
+    ws, d = ctypes.c_void_p(16), ctypes.c_void_p(16)
+    big = (1 << 30) + 64
+    for (M, N, K, want) in [(big, 128, 64, 10), (128, big, 64, 10), (128, 128, big - 32, 10),
+                            (0, 128, 64, 3), (128, 0, 64, 3), (128, 128, 0, 3)]:
+        a = nv.CTensor(16, 16, 0, 16, M, K, 0, 0)
+        b = nv.CTensor(16, 16, 0, 16, N, K, 0, 0)
+        assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, max(N, 8), 0, ws, None) == want, (M, N, K)
