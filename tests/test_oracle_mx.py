@@ -118,3 +118,15 @@ def test_sr_unbiased_per_element(ora):
     mean = (q * s).mean(axis=0)
     sd = (q * s).std(axis=0) / np.sqrt(rows) + 1e-12
     assert np.all(np.abs(mean - vals.astype(np.float64)) <= 4 * sd + 2.0 ** -16 * np.abs(vals))
+
+
+def test_hand_worked_block(ora):
+    # amax 3 -> floor(log2 3) = 1 -> E = -1, scale code 126, u = 2 v:
+    #   3.0 -> u = 6 -> code 7;   -1.25 -> u = -2.5, a tie between 2 and 3 -> the even code 4
+    #   (value 2), sign -> 0xC;   bf16(0.6) = 0.6015625 -> u = 1.203 -> nearest 1 -> code 2;
+    #   bf16(0.1) = 0.10009765625 -> u = 0.2002 < 0.25 -> 0;   zeros -> 0
+    v = np.zeros(32, np.float32)
+    v[:4] = [3.0, -1.25, 0.6015625, 0.10009765625]
+    codes, scales = ora.quantize_mx(_bits(v)[None, :])
+    assert scales.tolist() == [[126]]
+    assert codes[0, 0] == 0xC7 and codes[0, 1] == 0x02 and not codes[0, 2:].any()
