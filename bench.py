@@ -239,30 +239,72 @@ def run_ours(args, rank, world, local_rank):
         h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
         d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
 
+        # Host-to-device copies, compute and device-to-host copies on three streams, ordered by
+        # events so the two copy directions (PCIe is full duplex) overlap each other and the
+        # compute: step k's uploads wait for step k-1's compute to finish reading x, w and dy;
+        # its forward waits for x and w and for step k-1's read-back of y; its backward for dy
+        # and for step k-1's read-back of dx and dw; each read-back waits for its result.
+        comp = torch.cuda.current_stream(dev)
+        up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        evt = lambda: torch.cuda.Event()  # noqa: E731
+        prev = {"bwd": None, "y_read": None, "dxdw_read": None}
+
         def e2e_step(seed):
-            x.copy_(hx, non_blocking=True)
-            w.copy_(hw, non_blocking=True)
-            dy.copy_(hdy, non_blocking=True)
+            with torch.cuda.stream(up_s):
+                if prev["bwd"] is not None:
+                    up_s.wait_event(prev["bwd"])
+                x.copy_(hx, non_blocking=True)
+                w.copy_(hw, non_blocking=True)
+                xw_in = evt()
+                xw_in.record(up_s)
+                dy.copy_(hdy, non_blocking=True)
+                dy_in = evt()
+                dy_in.record(up_s)
+            comp.wait_event(xw_in)
+            if prev["y_read"] is not None:
+                comp.wait_event(prev["y_read"])
             nv.nvfp4_linear_fwd(ctx, x, w, y)
+            y_done = evt()
+            y_done.record(comp)
+            comp.wait_event(dy_in)
+            if prev["dxdw_read"] is not None:
+                comp.wait_event(prev["dxdw_read"])
             nv.nvfp4_linear_bwd(ctx, dy, seed, dx, dw)
-            hy.copy_(y, non_blocking=True)
-            hdx.copy_(dx, non_blocking=True)
-            hdw.copy_(dw, non_blocking=True)
+            bwd_done = evt()
+            bwd_done.record(comp)
+            with torch.cuda.stream(down_s):
+                down_s.wait_event(y_done)
+                hy.copy_(y, non_blocking=True)
+                y_read = evt()
+                y_read.record(down_s)
+                down_s.wait_event(bwd_done)
+                hdx.copy_(dx, non_blocking=True)
+                hdw.copy_(dw, non_blocking=True)
+                dxdw_read = evt()
+                dxdw_read.record(down_s)
+            prev.update(bwd=bwd_done, y_read=y_read, dxdw_read=dxdw_read)
 
         e2e_step(0)
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(comp)
+        up_s.wait_event(e0)                      # the first upload starts inside the timed region
         for k in range(args.e2e_steps):
             e2e_step(k)
-        e1.record()
+        comp.wait_event(prev["dxdw_read"])      # the last read-back ends the timed region
+        comp.wait_event(prev["y_read"])
+        e1.record(comp)
         torch.cuda.synchronize()
+        # the read-backs hold the last step's results
+        if not (torch.equal(hy, y.cpu()) and torch.equal(hdx, dx.cpu()) and torch.equal(hdw, dw.cpu())):
+            raise RuntimeError("end-to-end read-back differs from the device results")
         e2e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / args.e2e_steps
         e2e = {"value": job_tflops(world, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW"}
+               "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW; uploads, "
+                       "compute and read-backs on three event-ordered streams"}
 
     if rank != 0:
         return None
