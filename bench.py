@@ -36,9 +36,13 @@ FLOP_GEMM = 2 * T_TOK * D_IN * D_OUT
 Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FP4_OVER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+FP4_DENSE_DATASHEET_TFLOPS = 9000.0
+# tcgen05 block-scaled FP4 instruction rate: 16384 dense FP4 FMA per clock per SM (measured on
+# this GPU: four 128x256x64 MMAs take 512 cycles), 148 SMs
+FP4_FLOP_PER_CLK = 2 * 16384 * 148
 # DRAM bytes (read + write) per GEMM launch, the mean over the fprop, dgrad and wgrad launches
-# of one ncu capture (profiles/gemm_nvf4_2sm_kernel_8192x5120x20480.md), valid for the GEMM
-# source it was taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
+# of one ncu capture of the SM-pair GEMM at this layer's shapes, valid for the GEMM source it was
+# taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
 GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
 GEMM_TRAFFIC = {"sha256": "1b1ff1cb88ee135cae6fadffa2b5882b18ff9143af5e688ab53806a543826b35",
                 "bytes_per_launch": 486.5e6}
@@ -171,28 +175,30 @@ def run_ours(args, rank, world, local_rank):
     dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
-    # Per-call events: the step is the sequence of the library's public calls that
-    # nvfp4_linear_fwd / nvfp4_linear_bwd make, timed one by one on the current stream.
-    def step(sr_seed, ev=None):
-        def rec(i):
-            if ev is not None:
-                ev[i].record()
-        rec(0)
-        nv.nvfp4_quantize_weight(w, out=ctx.wq, out_t=ctx.wqt, ws=ctx.ws)
-        rec(1)
+    # The step as a user runs it: the two public entry points of the linear layer.
+    def step(sr_seed):
+        nv.nvfp4_linear_fwd(ctx, x, w, y)
+        nv.nvfp4_linear_bwd(ctx, dy, sr_seed, dx, dw)
+
+    # The same step as the sequence of public calls that nvfp4_linear_fwd / nvfp4_linear_bwd
+    # make, with an event between calls: the per-kernel fields (roofline, quantize, per-GEMM).
+    def step_calls(sr_seed, ev):
+        ev[0].record()
         nv.nvfp4_quantize_dual(x, mode=nv.RNE, rht_seed=0, out_row=ctx.xq, out_col=ctx.xq_rht, ws=ctx.ws)
-        rec(2)
+        ev[1].record()
+        nv.nvfp4_quantize_weight(w, out=ctx.wq, out_t=ctx.wqt, ws=ctx.ws)
+        ev[2].record()
         nv.nvfp4_gemm(ctx.xq, ctx.wq, out=y, ws=ctx.ws)
-        rec(3)
+        ev[3].record()
         nv.nvfp4_quantize_dual(dy, mode=nv.SR, rht_seed=0, sr_seed=sr_seed, stream_row=nv.STREAM_DGRAD,
                                stream_col=nv.STREAM_WGRAD, out_row=ctx.dyq, out_col=ctx.dyq_rht, ws=ctx.ws)
-        rec(4)
+        ev[4].record()
         nv.nvfp4_gemm(ctx.dyq, ctx.wqt, out=dx, ws=ctx.ws)
-        rec(5)
+        ev[5].record()
         nv.nvfp4_gemm(ctx.dyq_rht, ctx.xq_rht, out=dw, ws=ctx.ws)
-        rec(6)
+        ev[6].record()
 
-    launches_per_step = 2 + 2 + 1 + 2 + 1 + 1   # amax+tile (W), amax+tile (X), fprop, amax+tile (dY), dgrad, wgrad
+    launches_per_step = 2 + 2 + 1 + 2 + 1 + 1   # amax+tile (X), amax+tile (W), fprop, amax+tile (dY), dgrad, wgrad
 
     for i in range(args.warmup):
         step(1000 + i)
@@ -201,32 +207,43 @@ def run_ours(args, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     with ClockSampler(local_rank) as clk:
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
         for k in range(args.steps):
             flush.fill_(k & 0xFF)                  # evict L2 between steps (outside the events)
-            step(k, events[k])
+            events[k][0].record()
+            step(k)
+            events[k][1].record()
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
     status = nv.nvfp4_poll(ctx.ws)
     if status != 0:
         raise RuntimeError(f"device status {status} during timing")
+    ms_per_step = reduce_max(sum(a.elapsed_time(b) for a, b in events), dist, dev) / args.steps
 
-    seg = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(6)] for k in range(args.steps)]
-    step_ms = [sum(s) for s in seg]
-    ms_per_step = reduce_max(sum(step_ms), dist, dev) / args.steps
+    # per-call breakdown (same inputs, same L2 flush between steps)
+    cev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        step_calls(k, cev[k])
+    torch.cuda.synchronize()
+    if nv.nvfp4_poll(ctx.ws) != 0:
+        raise RuntimeError("device status during the per-call breakdown")
+    seg = [[cev[k][i].elapsed_time(cev[k][i + 1]) for i in range(6)] for k in range(args.steps)]
+    calls_ms_per_step = statistics.mean(sum(s_) for s_ in seg)
 
-    gemm_ms = [s[i] for s in seg for i in (2, 4, 5)]
-    q_ms = sum(s[0] + s[1] + s[3] for s in seg)
+    gemm_ms = [s_[i] for s_ in seg for i in (2, 4, 5)]
+    q_ms = sum(s_[0] + s_[1] + s_[3] for s_ in seg)
     q_bytes = args.steps * Q_BYTES_PER_ELEM * (D_OUT * D_IN + T_TOK * D_IN + T_TOK * D_OUT)
     peaks, peak_kind = load_peaks()
     gemm_avg_ms = statistics.mean(gemm_ms)
     achieved = FLOP_GEMM / (gemm_avg_ms * 1e-3) / 1e12
-    peak_tensor = FP4_OVER_BF16 * peaks["bf16_tflops_sustained"]
+    # each GEMM launch is timed alone (a third of a ~2 ms step): the burst bf16 figure is its basis
+    peak_tensor = FP4_OVER_BF16 * peaks["bf16_tflops"]
     q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
 
     # ---- end to end through the public API from pinned host buffers ---------------------
@@ -306,8 +323,11 @@ def run_ours(args, rank, world, local_rank):
                "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW; uploads, "
                        "compute and read-backs on three event-ordered streams"}
 
+    ffn = ffn_fields(args, world, dev, dist, flush) if args.ffn else None
     if rank != 0:
         return None
+    clocks = clk.summary()
+    inst_peak = FP4_FLOP_PER_CLK * clocks["sm_mhz"] * 1e6 / 1e12 if clocks.get("sm_mhz") else None
     line = {
         "metric": METRIC,
         "value": job_tflops(world, ms_per_step),
@@ -325,22 +345,31 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_2sm_kernel", "achieved": achieved,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
                      "traffic": gemm_traffic(),
-                     "peak_basis": f"{FP4_OVER_BF16:g} x {peak_kind} sustained bf16 ({peaks['bf16_tflops_sustained']} TF/s)",
+                     "peak_basis": f"{FP4_OVER_BF16:g} x {peak_kind} burst bf16 ({peaks['bf16_tflops']} TF/s)",
+                     "frac_of_9pf_datasheet": achieved / FP4_DENSE_DATASHEET_TFLOPS,
+                     "frac_of_instruction_rate_at_clock": achieved / inst_peak if inst_peak else None,
                      "per_launch_flop": FLOP_GEMM, "avg_launch_ms": gemm_avg_ms},
         "quantize": {"gbs": q_gbs, "unit": "GB/s", "peak_hbm_gbs": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
                      "bytes_per_elem": Q_BYTES_PER_ELEM, "peak_basis": peak_kind,
-                     "per_call_ms": {"W": statistics.mean(s[0] for s in seg), "X": statistics.mean(s[1] for s in seg),
-                                     "dY": statistics.mean(s[3] for s in seg)}},
-        "gemm_tflops": {"fprop": FLOP_GEMM / statistics.mean(s[2] for s in seg) / 1e9,
-                        "dgrad": FLOP_GEMM / statistics.mean(s[4] for s in seg) / 1e9,
-                        "wgrad": FLOP_GEMM / statistics.mean(s[5] for s in seg) / 1e9},
-        "clocks": clk.summary(),
+                     "per_call_ms": {"X": statistics.mean(s_[0] for s_ in seg), "W": statistics.mean(s_[1] for s_ in seg),
+                                     "dY": statistics.mean(s_[3] for s_ in seg)},
+                     "per_call_gbs": {
+                         "X": Q_BYTES_PER_ELEM * T_TOK * D_IN / statistics.mean(s_[0] for s_ in seg) / 1e6,
+                         "W": Q_BYTES_PER_ELEM * D_OUT * D_IN / statistics.mean(s_[1] for s_ in seg) / 1e6,
+                         "dY": Q_BYTES_PER_ELEM * T_TOK * D_OUT / statistics.mean(s_[3] for s_ in seg) / 1e6}},
+        "gemm_tflops": {"fprop": FLOP_GEMM / statistics.mean(s_[2] for s_ in seg) / 1e9,
+                        "dgrad": FLOP_GEMM / statistics.mean(s_[4] for s_ in seg) / 1e9,
+                        "wgrad": FLOP_GEMM / statistics.mean(s_[5] for s_ in seg) / 1e9},
+        "calls_ms_per_step": calls_ms_per_step,
+        "clocks": clocks,
         "e2e": e2e,
+        "c1_small_fprop": c1_latency(nv, dev),
+        "ffn_step": ffn,
         "gpu_launches": launches_per_step * args.steps,
         "impl": "ours",
     }
     if args.cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args)
+        line["cpu_baseline"] = cpu_baseline_with_one_core(args)
     return line
 
 
@@ -352,70 +381,108 @@ FFN_T, FFN_D, FFN_F = 16384, 5120, 20480
 FFN_FLOP = 6 * 2 * FFN_T * FFN_D * FFN_F
 
 
+class FFNStep:
+    """The one-FFN training step on one rank's batch, its buffers allocated once."""
+
+    def __init__(self, nv, dev):
+        import synth
+        self.nv = nv
+        self.x = synth.activations(FFN_T, FFN_D, seed=0, outlier_frac=0.001).to(dev)
+        self.w1 = synth.weights(FFN_F, FFN_D, seed=1).to(dev)
+        self.w2 = synth.weights(FFN_D, FFN_F, seed=3).to(dev)
+        self.dy = synth.grad_output(FFN_T, FFN_D, seed=4).to(dev)
+        self.up = nv.LinearContext(FFN_T, FFN_D, FFN_F, rht_seed=0, device=dev)
+        self.down = nv.LinearContext(FFN_T, FFN_F, FFN_D, rht_seed=0, device=dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        self.h, self.g, self.dg, self.dh = (torch.empty((FFN_T, FFN_F), **bf) for _ in range(4))
+        self.y, self.dx = torch.empty((FFN_T, FFN_D), **bf), torch.empty((FFN_T, FFN_D), **bf)
+        self.dw1 = torch.empty((FFN_F, FFN_D), dtype=torch.float32, device=dev)
+        self.dw2 = torch.empty((FFN_D, FFN_F), dtype=torch.float32, device=dev)
+
+    @staticmethod
+    def launches_per_step(fused: bool) -> int:
+        # 2 x (W quantize 2 + X/G quantize 2 + fprop 1) + 2 x (dY/dH quantize 2 + dgrad 1 + wgrad 1)
+        # + 2 GeLU; the fused variant drops the amax passes of G and dH
+        return 2 * 5 + 2 * 4 + 2 - (2 if fused else 0)
+
+    def step(self, seed: int, fused: bool):
+        nv = self.nv
+        nv.nvfp4_linear_fwd(self.up, self.x, self.w1, self.h)
+        if fused:   # the GeLU kernels reduce their output's amax; G's and dH's quantize skip pass 1
+            nv.nvfp4_gelu_fwd_amax(self.h, self.g, rht_seed=0, ws=self.down.ws)
+            self.down.amax_ready = True
+        else:
+            nv.nvfp4_gelu_fwd(self.h, self.g)
+        nv.nvfp4_linear_fwd(self.down, self.g, self.w2, self.y)
+        nv.nvfp4_linear_bwd(self.down, self.dy, 2 * seed, self.dg, self.dw2)
+        if fused:
+            nv.nvfp4_gelu_bwd_amax(self.h, self.dg, self.dh, rht_seed=0, ws=self.up.ws)
+            self.up.amax_ready = True
+        else:
+            nv.nvfp4_gelu_bwd(self.h, self.dg, self.dh)
+        nv.nvfp4_linear_bwd(self.up, self.dh, 2 * seed + 1, self.dx, self.dw1)
+
+    def poll(self, what: str):
+        for c in (self.up, self.down):
+            if self.nv.nvfp4_poll(c.ws) != 0:
+                raise RuntimeError(f"device status {what}")
+
+    def time(self, steps, warmup, fused, flush, dist, dev, clk_gpu=None):
+        """ms per step (max over ranks) and the clock summary of the timed region."""
+        for i in range(warmup):
+            self.step(1000 + i, fused)
+        torch.cuda.synchronize()
+        self.poll("after warm-up")
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with ClockSampler(clk_gpu if clk_gpu is not None else dev.index) as clk:
+            if dist:
+                dist.barrier()
+            torch.cuda.synchronize()
+            for k in range(steps):
+                flush.fill_(k & 0xFF)                  # evict L2 between steps (outside the events)
+                ev[k][0].record()
+                self.step(k, fused)
+                ev[k][1].record()
+            torch.cuda.synchronize()
+            if dist:
+                dist.barrier()
+        self.poll("during timing")
+        return reduce_max(sum(a.elapsed_time(b) for a, b in ev), dist, dev) / steps, clk.summary()
+
+
+def ffn_config(fused: bool) -> dict:
+    return {"workload": "one FFN training step: up 5120->20480, GeLU, down 20480->5120, forward and "
+                        "backward (6 GEMMs), weights quantized every step"
+                        + (", amax of G and dH fused into the GeLU kernels" if fused else ""),
+            "tokens": FFN_T, "d": FFN_D, "ffn": FFN_F, "flop_per_step": FFN_FLOP,
+            "l2": "256 MiB buffer written between timed steps (outside the events)"}
+
+
+def ffn_fields(args, world, dev, dist, flush) -> dict:
+    """The FFN step, plain and with the GeLU-fused amax, as a nested field of the main line."""
+    import nvfp4_bit_quantized_02_b200 as nv
+    f = FFNStep(nv, dev)
+    out = {}
+    for fused in (False, True):
+        ms, clocks = f.time(args.steps, args.warmup, fused, flush, dist, dev)
+        out["fused_amax" if fused else "plain"] = {
+            "value": world * FFN_FLOP / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms,
+            "gpu_launches": f.launches_per_step(fused) * args.steps, "clocks": clocks, "config": ffn_config(fused)}
+    del f
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ffn(args, rank, world, local_rank):
     import nvfp4_bit_quantized_02_b200 as nv
-    import synth
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     dist = torch.distributed if world > 1 else None
-    x = synth.activations(FFN_T, FFN_D, seed=0, outlier_frac=0.001).to(dev)
-    w1 = synth.weights(FFN_F, FFN_D, seed=1).to(dev)
-    w2 = synth.weights(FFN_D, FFN_F, seed=3).to(dev)
-    dy = synth.grad_output(FFN_T, FFN_D, seed=4).to(dev)
-    up = nv.LinearContext(FFN_T, FFN_D, FFN_F, rht_seed=0, device=dev)
-    down = nv.LinearContext(FFN_T, FFN_F, FFN_D, rht_seed=0, device=dev)
-    bf = dict(dtype=torch.bfloat16, device=dev)
-    h, g, dg, dh = (torch.empty((FFN_T, FFN_F), **bf) for _ in range(4))
-    y, dx = torch.empty((FFN_T, FFN_D), **bf), torch.empty((FFN_T, FFN_D), **bf)
-    dw1 = torch.empty((FFN_F, FFN_D), dtype=torch.float32, device=dev)
-    dw2 = torch.empty((FFN_D, FFN_F), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
     fused = args.ffn_fused_amax
-
-    def step(seed):
-        nv.nvfp4_linear_fwd(up, x, w1, h)
-        if fused:   # the GeLU kernels reduce their output's amax; G's and dH's quantize skip pass 1
-            nv.nvfp4_gelu_fwd_amax(h, g, rht_seed=0, ws=down.ws)
-            down.amax_ready = True
-        else:
-            nv.nvfp4_gelu_fwd(h, g)
-        nv.nvfp4_linear_fwd(down, g, w2, y)
-        nv.nvfp4_linear_bwd(down, dy, 2 * seed, dg, dw2)
-        if fused:
-            nv.nvfp4_gelu_bwd_amax(h, dg, dh, rht_seed=0, ws=up.ws)
-            up.amax_ready = True
-        else:
-            nv.nvfp4_gelu_bwd(h, dg, dh)
-        nv.nvfp4_linear_bwd(up, dh, 2 * seed + 1, dx, dw1)
-
-    # per step: 2 x (W quantize 2 + X/G quantize 2 + fprop 1) + 2 x (dY/dH quantize 2 + dgrad 1
-    # + wgrad 1) + 2 GeLU; the fused variant drops the amax passes of G and dH
-    launches_per_step = 2 * 5 + 2 * 4 + 2 - (2 if fused else 0)
-    for i in range(args.warmup):
-        step(1000 + i)
-    torch.cuda.synchronize()
-    for c in (up, down):
-        if nv.nvfp4_poll(c.ws) != 0:
-            raise RuntimeError("device status after warm-up")
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    with ClockSampler(local_rank) as clk:
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize()
-        for k in range(args.steps):
-            flush.fill_(k & 0xFF)                  # evict L2 between steps (outside the events)
-            ev[k][0].record()
-            step(k)
-            ev[k][1].record()
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
-    for c in (up, down):
-        if nv.nvfp4_poll(c.ws) != 0:
-            raise RuntimeError("device status during timing")
-    ms_per_step = reduce_max(sum(a.elapsed_time(b) for a, b in ev), dist, dev) / args.steps
+    f = FFNStep(nv, dev)
+    ms_per_step, clocks = f.time(args.steps, args.warmup, fused, flush, dist, dev)
     if rank != 0:
         return None
     return {
@@ -431,33 +498,67 @@ def run_ffn(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate; GeLU fp32 math, bf16 in/out",
         "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W1 and W2, N(0,1e-4) dY; bf16)",
-        "config": {"workload": "one FFN training step: up 5120->20480, GeLU, down 20480->5120, forward and "
-                               "backward (6 GEMMs), weights quantized every step"
-                               + (", amax of G and dH fused into the GeLU kernels" if fused else ""),
-                   "tokens": FFN_T, "d": FFN_D, "ffn": FFN_F, "flop_per_step": FFN_FLOP,
-                   "l2": "256 MiB buffer written between timed steps (outside the events)"},
-        "clocks": clk.summary(),
+        "config": ffn_config(fused),
+        "clocks": clocks,
         "e2e": None,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": f.launches_per_step(fused) * args.steps,
         "impl": "ours",
     }
+
+
+def c1_latency(nv, dev) -> dict:
+    """The 256 x 256 x 256 fprop of the small single-GEMM workload, reported as latency: the GEMM
+    launch alone and the whole fprop (both quantize calls + GEMM), median over back-to-back
+    repetitions (the operands are L2-resident; a latency, not a bandwidth figure)."""
+    import synth
+    x = synth.activations(256, 256, seed=0).to(dev)
+    w = synth.weights(256, 256, seed=1).to(dev)
+    ws = nv.Workspace(dev)
+    xq = nv.nvfp4_quantize(x, ws=ws)
+    wq = nv.nvfp4_quantize(w, block=nv.BLOCK_16x16, ws=ws)
+    y = torch.empty((256, 256), dtype=torch.bfloat16, device=dev)
+
+    def fprop():
+        nv.nvfp4_quantize(x, out=xq, ws=ws)
+        nv.nvfp4_quantize(w, block=nv.BLOCK_16x16, out=wq, ws=ws)
+        nv.nvfp4_gemm(xq, wq, out=y, ws=ws)
+
+    res = {}
+    for name, fn in (("gemm_us", lambda: nv.nvfp4_gemm(xq, wq, out=y, ws=ws)), ("fprop_us", fprop)):
+        for _ in range(20):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(200):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        res[name] = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+    if nv.nvfp4_poll(ws) != 0:
+        raise RuntimeError("device status in the small fprop")
+    res["workload"] = "fprop 256x256x256: X N(0,1) 1x16 RNE, W N(0,0.02) 16x16 RNE, bf16 out"
+    return res
 
 
 # ---------------------------------------------------------------------------------------
 # the CPU oracle (reference arm and the cpu_baseline field)
 # ---------------------------------------------------------------------------------------
-def cpu_baseline(args, n_cols: int | None = None):
+def cpu_baseline(args, n_cols: int | None = None, threads: int | None = None):
     """The oracle as it stands on a bounded slice of the same layer: the first T_s tokens and the
     first n_s output features with the full d = 5120 (all six quantized forms, the three GEMMs
-    over every output of the slice)."""
+    over every output of the slice), on `threads` host threads (all cores by default).  The
+    default slice is sized for about 10 s of oracle work."""
     import numpy as np
 
     import oracle
     import synth
 
-    cores = os.cpu_count() or 1
+    cores = threads or os.cpu_count() or 1
     T_s = 256
-    n_s = n_cols or min(D_OUT, 4096 * max(1, cores // 8))   # about 10 s of oracle work
+    n_s = n_cols or min(D_OUT, 4096 * max(1, cores // 8))   # about 10 s of oracle work on all cores
     x = synth.bf16_bits(synth.activations(T_TOK, D_IN, seed=0, outlier_frac=0.001)[:T_s])
     w = synth.bf16_bits(synth.weights(D_OUT, D_IN, seed=1)[:n_s])
     dy = synth.bf16_bits(synth.grad_output(T_TOK, D_OUT, seed=2)[:T_s, :n_s])
@@ -481,6 +582,16 @@ def cpu_baseline(args, n_cols: int | None = None):
     return {"value": flop / dt / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "seconds": dt,
             "sample": f"layer slice T={T_s} tokens x n={n_s} out-features x d={D_IN}: six quantized forms and the "
                       f"fprop/dgrad/wgrad GEMMs (fp64 over dequantized operands) of the slice, {flop / 1e9:.1f} GFLOP"}
+
+
+def cpu_baseline_with_one_core(args):
+    """All host cores (the reported value) and, beside it, one core on a 16x smaller slice (the
+    oracle is scalar code: one core is its plain speed)."""
+    n_all = min(D_OUT, 4096 * max(1, (os.cpu_count() or 1) // 8))
+    allc = cpu_baseline(args, n_cols=n_all)
+    one = cpu_baseline(args, n_cols=max(256, n_all // 16), threads=1)
+    allc["one_core"] = {k: one[k] for k in ("value", "unit", "cores", "seconds", "sample")}
+    return allc
 
 
 def run_reference(args, rank, world):
@@ -513,6 +624,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--workload", choices=["linear", "ffn"], default="linear",
                     help="linear: the 8192x5120x20480 layer (the default line); ffn: the one-FFN step")
+    ap.add_argument("--no-ffn", dest="ffn", action="store_false",
+                    help="linear: skip the nested one-FFN step fields")
     ap.add_argument("--ffn-fused-amax", action="store_true",
                     help="ffn: the GeLU kernels that also reduce their output's amax (slower as they stand)")
     args = ap.parse_args()

@@ -244,13 +244,20 @@ nvfp4_status nvfp4_gelu_bwd_amax(const void* h, const void* dg, void* dh, int64_
  * Its 256-byte scratch is a fixed device array inside the library, held by every GPU that
  * loads the library until the process exits; a call whose scratch would not fit returns
  * NVFP4_ERR_LIMIT.  The first call on a device looks up the array's device address (do it
- * before any stream capture).  All calls share the array, so calls that overlap on the GPU
- * race; serialise them.  Non-finite inputs are not reported by this variant.
+ * before any stream capture); that address does not survive cudaDeviceReset of the device.
+ * All calls share the array, so calls that overlap on the GPU race; serialise them.
+ * Device-side conditions (non-finite input, a wait that ran out of its budget) are kept in the
+ * array until nvfp4_poll_noalloc reports them; the output of a flagged call is undefined.
  */
 nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along,
                                     nvfp4_round mode, nvfp4_block block, int rht, uint64_t rht_seed,
                                     uint64_t sr_seed, uint32_t stream_id, nvfp4_tensor* out,
                                     nvfp4_stream_t stream);
+
+/* nvfp4_poll for nvfp4_quantize_noalloc (no counterpart in the pages either): synchronize
+ * `stream`, then report and clear the flags that the workspace-free calls on the current
+ * device left in the library's array, with the precedence of nvfp4_poll.  Allocates nothing. */
+nvfp4_status nvfp4_poll_noalloc(nvfp4_stream_t stream);
 
 /* Synchronize `stream`, then report (and clear) the device flags of `ws`: NVFP4_ERR_TIMEOUT
  * takes precedence over NVFP4_ERR_NONFINITE; NVFP4_OK when neither is set. */

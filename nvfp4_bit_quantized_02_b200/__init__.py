@@ -84,6 +84,8 @@ def _lib():
             "nvfp4_gelu_fwd_amax": ([vp, vp, i64, i64, u64, vp, vp], i32),
             "nvfp4_gelu_bwd_amax": ([vp, vp, vp, i64, i64, u64, vp, vp], i32),
             "nvfp4_poll": ([vp, vp], i32),
+            "nvfp4_quantize_noalloc": ([vp, i64, i64, i64, i32, i32, i32, i32, u64, u64, u32, T, vp], i32),
+            "nvfp4_poll_noalloc": ([vp], i32),
             "nvfp4_set_wait_budget_ns": ([u64], None),
             "nvfp4_status_string": ([i32], c.c_char_p),
             "nvfp4_version": ([], i32),

@@ -69,6 +69,11 @@ static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
 // N >> 3 at bit 17, scale type UE4M3 (bit 23 = 0), M >> 4 at bit 24, scale ids 0
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 
+// Budget of the teardown waits (copies and MMAs still in flight after an abort).  Fixed, not the
+// caller's budget: however small that is, no CTA exits (or frees TMEM) before its own copies have
+// landed and its MMAs have completed.
+constexpr uint64_t kDrainBudgetNs = 2000000000ull;
+
 // ---------------------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------------------
@@ -414,12 +419,12 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
                     }
                 }
             }
-            if (*abort_flag) {
-                // drain: every copy this thread issued must land before the CTA exits
-                for (int k = max(0, g - kStages); k < g; ++k)
-                    mbar_wait(smem_u32(&full_bar[k % kStages]), (uint32_t)(k / kStages) & 1u, abort_flag, p.flags,
-                              p.budget_ns, false);
-            }
+            // drain: every copy this thread issued lands before the CTA exits.  Stages before
+            // g - kStages were consumed (their slots were refilled); after a normal run the last
+            // kStages were consumed too and these waits return at once.
+            for (int k = max(0, g - kStages); k < g; ++k)
+                mbar_wait(smem_u32(&full_bar[k % kStages]), (uint32_t)(k / kStages) & 1u, abort_flag, p.flags,
+                          kDrainBudgetNs, false);
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -----------------------------------------
@@ -465,7 +470,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         // all MMAs of this warp complete before TMEM may be freed
         if (elect_one()) mma_commit(smem_u32(done_bar));
         __syncwarp();
-        mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+        mbar_wait(smem_u32(done_bar), 0u, abort_flag, p.flags, kDrainBudgetNs, false);
     } else if (warp < 2 + kEpi1Warps) {
         // ------------------------------- epilogue (warps 2..17) -----------------------------
         // Each warp owns 32 accumulator rows (its TMEM lane quadrant) x 64 columns.  It reads
@@ -658,6 +663,15 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 __device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+// cancel `bytes` of a barrier phase's expected transaction count (copies that were never issued)
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -679,6 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     uint64_t* edrained_bar = boxgo_bar + 2 * kEpi1Warps;                  // peer: its epilogue drained
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(edrained_bar + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
+    uint32_t* issued_slot = tmem_slot + 2;                                // stages this CTA's producer issued
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -741,12 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
                     tma_load_2d_pair(smem_u32(st + k2CodeBytes + kSFABytes), &tmSB, kb * 256, tn * 2, full_leader);
                 }
             }
-            if (*abort_flag && rank == 0) {
-                // the leader's barrier counts both CTAs' bytes: the peer's copies land on it too
-                for (int k = max(0, g - k2Stages); k < g; ++k)
-                    mbar_wait_cl(smem_u32(&full_bar[k % k2Stages]), (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags,
-                                 p.budget_ns, false);
-            }
+            *issued_slot = (uint32_t)g;   // read by the leader's drain after the first cluster barrier
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer (leader only) ----------------------------
@@ -796,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             }
             if (elect_one()) mma_commit_local_pair(smem_u32(done_bar));
             __syncwarp();
-            mbar_wait_cl(smem_u32(done_bar), 0u, abort_flag, p.flags, p.budget_ns, false);
+            mbar_wait_cl(smem_u32(done_bar), 0u, abort_flag, p.flags, kDrainBudgetNs, false);
         } else {
             // The peer's MMA warp forwards its CTA's drained accumulator to the leader as one
             // remote arrival per tile, so the epilogue warps arrive locally (cheap) and one remote
@@ -843,6 +853,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     }
 
     tc_fence_before();
+    cluster_sync_all();   // both producers have stopped issuing and published their stage counts
+    if (warp == 0 && lane == 0 && rank == 0) {
+        // Drain: every copy of either CTA lands before either exits.  All copies of a stage land on
+        // the leader's full barrier, so the leader waits there for the stages that may still be
+        // outstanding.  A producer cannot run more than k2Stages ahead of the slower one (a slot is
+        // refilled only after the MMAs consumed it, which needs both CTAs' copies), so those are
+        // the last k2Stages before the larger count, one phase per barrier.  After an abort the
+        // two counts can differ: a stage only the peer issued has its missing arrival made here
+        // (for the peer's bytes); a stage only the leader issued has the peer's bytes cancelled.
+        // After a normal run both counts are equal, all stages were consumed, and every wait
+        // returns at once.
+        const int gl = (int)*issued_slot;
+        const int gp = (int)ld_cluster_u32(map_rank(smem_u32(issued_slot), 1));
+        const int gmax = max(gl, gp);
+        for (int k = max(0, gmax - k2Stages); k < gmax; ++k) {
+            const uint32_t bar = smem_u32(&full_bar[k % k2Stages]);
+            if (k >= gl)
+                mbar_expect_tx(bar, (uint32_t)k2StageBytes);
+            else if (k >= gp)
+                mbar_complete_tx(bar, (uint32_t)k2StageBytes);
+            mbar_wait_cl(bar, (uint32_t)(k / k2Stages) & 1u, abort_flag, p.flags, kDrainBudgetNs, false);
+        }
+    }
     cluster_sync_all();   // both CTAs finished with TMEM, barriers and each other's shared memory
     if (warp == 1) {
         tc_fence_after();

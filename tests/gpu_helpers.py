@@ -86,6 +86,31 @@ def check_gemm(d_gpu: np.ndarray, d_ref: np.ndarray, sabs: np.ndarray, bf16_out:
                              f"gpu {d_gpu.reshape(-1)[i]!r} ref {d_ref.reshape(-1)[i]!r} tol {np.reshape(tol, -1)[i]!r}")
 
 
+def sample_positions(Mo: int, No: int, seed: int):
+    """Output positions checked at full size: every element of 8 full 128 x 128 tiles (the four
+    corners, the centre and three seeded random tiles) plus 65536 seeded random elements."""
+    tiles = [(0, 0), (0, No // 128 - 1), (Mo // 128 - 1, 0), (Mo // 128 - 1, No // 128 - 1),
+             (Mo // 256, No // 256)]
+    rng = np.random.default_rng(seed)
+    tiles += [(int(rng.integers(0, Mo // 128)), int(rng.integers(0, No // 128))) for _ in range(3)]
+    ii, jj = [], []
+    for ti, tj in tiles:
+        a, b = np.meshgrid(np.arange(128) + 128 * ti, np.arange(128) + 128 * tj, indexing="ij")
+        ii.append(a.reshape(-1))
+        jj.append(b.reshape(-1))
+    ri, rj = synth.sample_indices(Mo, No, 65536, seed)
+    return np.concatenate(ii + [ri]), np.concatenate(jj + [rj])
+
+
+def check_gemm_sampled(out: torch.Tensor, a: "oracle.QForm", b: "oracle.QForm", bf16_out: bool, what: str, seed: int):
+    """A GEMM output checked on sample_positions against the oracle's fp64 GEMM."""
+    Mo, No = out.shape
+    ii, jj = sample_positions(Mo, No, seed)
+    ref, s = oracle.gemm_sampled(a, b, ii, jj)
+    got = out[torch.from_numpy(ii).to(out.device), torch.from_numpy(jj).to(out.device)]
+    check_gemm(bf16_to_f64(got) if bf16_out else got.cpu().numpy().astype(np.float64), ref, s, bf16_out, what)
+
+
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 

@@ -134,3 +134,15 @@ def test_e2m1_sr_codes_at_every_threshold():
                     parallel_map(work, range(0, n, step))
                     bad = np.nonzero(got != want)[0]
                     assert bad.size == 0, f"u={xs[bad[0]]!r} r={r[bad[0]]}: gpu {got[bad[0]]} oracle {want[bad[0]]}"
+
+
+@pytest.mark.parametrize("seed", [0, 7, 0x123456789ABCDEF, 2 ** 64 - 1])
+def test_rht_signs_are_the_low_half_of_curands_block_at_stream_3(seed):
+    # The RHT sign word is the low 16 bits of word 0 of the Philox4x32-10 block at counter
+    # (0, 0, 3, 0) under the seed: computed here by cuRAND's own Philox4_32_10 (subsequence 3,
+    # offset 0), an implementation the oracle shares nothing with.
+    L = checks()
+    cur = torch.empty(4, dtype=torch.int32, device="cuda")
+    assert L.chk_curand_philox(seed, 3, 0, 1, ctypes.c_void_p(cur.data_ptr())) == 0
+    word0 = int(cur.cpu().numpy().view(np.uint32)[0])
+    assert oracle.rht_signs(seed) == word0 & 0xFFFF

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import assert_form_equal, bf16_to_f64, check_gemm, nv, to_device_bf16
+from gpu_helpers import assert_form_equal, bf16_to_f64, check_gemm, check_gemm_sampled, nv, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -53,20 +53,6 @@ def test_small_layer_full_check(T, d, n):
     check_gemm(dw.cpu().numpy(), ref, s, False, "wgrad")
 
 
-def _sample(Mo, No, seed):
-    tiles = [(0, 0), (0, No // 128 - 1), (Mo // 128 - 1, 0), (Mo // 128 - 1, No // 128 - 1),
-             (Mo // 256, No // 256)]
-    rng = np.random.default_rng(seed)
-    tiles += [(int(rng.integers(0, Mo // 128)), int(rng.integers(0, No // 128))) for _ in range(3)]
-    ii, jj = [], []
-    for ti, tj in tiles:
-        a, b = np.meshgrid(np.arange(128) + 128 * ti, np.arange(128) + 128 * tj, indexing="ij")
-        ii.append(a.reshape(-1))
-        jj.append(b.reshape(-1))
-    ri, rj = synth.sample_indices(Mo, No, 65536, seed)
-    return np.concatenate(ii + [ri]), np.concatenate(jj + [rj])
-
-
 def test_full_size_layer_sampled():
     T, d, n = synth.TOKENS, synth.D_IN, synth.D_OUT
     x = synth.activations(T, d, seed=0, outlier_frac=0.001)
@@ -78,11 +64,7 @@ def test_full_size_layer_sampled():
         assert_form_equal(getattr(ctx, name), o[name], name)
     for what, out, a, b, bf in (("fprop", y, "xq", "wq", True), ("dgrad", dx, "dyq", "wqt", True),
                                 ("wgrad", dw, "dyq_rht", "xq_rht", False)):
-        Mo, No = out.shape
-        ii, jj = _sample(Mo, No, seed={"fprop": 1, "dgrad": 2, "wgrad": 3}[what])
-        ref, s = oracle.gemm_sampled(o[a], o[b], ii, jj)
-        got = out[torch.from_numpy(ii).cuda(), torch.from_numpy(jj).cuda()]
-        check_gemm(bf16_to_f64(got) if bf else got.cpu().numpy().astype(np.float64), ref, s, bf, what)
+        check_gemm_sampled(out, o[a], o[b], bf, what, seed={"fprop": 1, "dgrad": 2, "wgrad": 3}[what])
 
 
 def test_cached_weight_path_identical():

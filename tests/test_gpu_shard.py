@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import assert_form_equal, make_form, nv, to_device_bf16
+from gpu_helpers import assert_form_equal, check_gemm, make_form, nv, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -73,3 +73,40 @@ def test_dp_helper_on_one_rank_equals_whole_tensor_call():
             assert torch.equal(a.tensor_scale, b.tensor_scale)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,d,n,shards", [(1024, 256, 384, 2), (1024, 320, 256, 4)])
+def test_shard_wgrad_partials_reduce_to_the_whole_batch_dw(T, d, n, shards):
+    # Data-parallel wgrad: with the amax reduced across ranks and SR indexed in the whole batch's
+    # forms, each rank's dW partial is GEMM(its K range of dY^T, its K range of X^T); the fp32 sum
+    # of the partials (what the ranks' reduction computes) equals the whole batch's dW within the
+    # GEMM bound |err| <= 1e-5 sum_k |a_k b_k|, the sum now running over all T tokens.
+    m = nv()
+    x = synth.activations(T, d, seed=0, outlier_frac=0.01)
+    dy = synth.grad_output(T, n, seed=2)
+    rht_seed, sr_seed = 3, 4
+    q_x = oracle.quantize(synth.bf16_bits(x), along=1, rht=True, rht_seed=rht_seed)
+    q_dy = oracle.quantize(synth.bf16_bits(dy), along=1, mode=oracle.SR, rht=True, rht_seed=rht_seed,
+                           sr_seed=sr_seed, stream_id=2)
+    ref, sabs = oracle.gemm_full(q_dy, q_x)
+    rows = T // shards
+
+    def shard_forms(t, mode):
+        parts = [to_device_bf16(t[i * rows:(i + 1) * rows]) for i in range(shards)]
+        wss = [m.Workspace() for _ in range(shards)]
+        for p, ws in zip(parts, wss):
+            m.nvfp4_amax(p, True, rht_seed, ws)
+        words = torch.stack([ws.amax_words() for ws in wss]).max(dim=0).values   # the ranks' MAX all-reduce
+        out = []
+        for i, (p, ws) in enumerate(zip(parts, wss)):
+            ws.amax_words().copy_(words)
+            _, c = m.nvfp4_quantize_dual_shard(p, i * rows, T, mode, rht_seed, sr_seed, 1, 2, ws=ws)
+            assert m.nvfp4_poll(ws) == 0
+            out.append(c)
+        return out
+
+    xc, dyc = shard_forms(x, 0), shard_forms(dy, 1)
+    total = torch.zeros((n, d), dtype=torch.float32, device="cuda")
+    for a, b in zip(dyc, xc):
+        total += m.nvfp4_gemm(a, b, out_dtype=torch.float32)
+    check_gemm(total.cpu().numpy(), ref, sabs, False, f"sum of {shards} shard dW partials")

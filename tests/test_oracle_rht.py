@@ -55,3 +55,39 @@ def test_signs_depend_on_seed(ora):
     s = {ora.rht_signs(seed) for seed in range(64)}
     assert len(s) > 50
     assert all(0 <= v < (1 << 16) for v in s)
+
+
+def test_every_sign_bit_is_a_fair_coin_over_seeds(ora):
+    # The pages call the rotation "random": each of the 16 diagonal signs must be +1 or -1 with
+    # probability 1/2 over seeds.  Over 10^4 seeds every bit's frequency lies within 4 sigma of
+    # 1/2 (sigma = 0.005), every pair of bits agrees about half the time, and the 16-bit words
+    # are nearly all distinct (a mask that kept 8 of the 16 bits, a stuck bit, or one word shared
+    # by both halves fails one of these).
+    n = 10000
+    words = np.array([ora.rht_signs(seed) for seed in range(n)], np.uint32)
+    bits = ((words[:, None] >> np.arange(16)) & 1).astype(np.float64)
+    freq = bits.mean(axis=0)
+    assert np.all(np.abs(freq - 0.5) < 4 * 0.005), freq
+    agree = (bits[:, :, None] == bits[:, None, :]).mean(axis=0)
+    off = agree[~np.eye(16, dtype=bool)]
+    assert np.all(np.abs(off - 0.5) < 4 * 0.005), off.min()
+    # 10^4 draws from 2^16 values: about 9.3e3 distinct in expectation
+    assert len(set(words.tolist())) > 9000
+
+
+@pytest.mark.parametrize("seed", [0, 5, 2 ** 40 + 3])
+def test_quantizer_rotates_with_the_signs_of_its_seed(ora, seed):
+    # The RHT form of a column holding one nonzero value e_j in a 16-token group has, in its
+    # 16 outputs, exactly 0.25 * s_j * H[:, j] times that value: the sign the quantizer applied
+    # to token j is read back from its codes and equals bit j of rht_signs(seed).
+    signs = ora.rht_signs(seed)
+    for j in range(16):
+        x = np.zeros((16, 16), np.uint16)
+        x[j, 0] = 0x3F80          # bf16 1.0 in column 0 at token j
+        q = ora.quantize(x, along=1, rht=True, rht_seed=seed)
+        nib = q.nibbles()[0]      # form row 0 = source column 0, K = the 16 tokens
+        # every output has magnitude 0.25 -> the block maximum, code 6.0 (0x7) with its sign
+        assert np.all((nib & 7) == 7), nib
+        got_sign = np.where(nib & 8, -1.0, 1.0)
+        sj = -1.0 if (signs >> j) & 1 else 1.0
+        assert np.array_equal(got_sign, sj * H16[:, j]), (j, got_sign)

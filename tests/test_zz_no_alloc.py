@@ -58,3 +58,50 @@ def test_noalloc_matches_workspace_entry_point(kind, along, mode, block, rht):
                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         assert st == 0, f"call {call}: status {st}"
         _same(nv, out, ref)
+
+
+def _call(nv, f, x, rows, cols, along, mode, block, rht, out):
+    ct = out.c()
+    xp = ctypes.c_void_p(x.data_ptr()) if x is not None and x.numel() else None
+    st = f(xp, rows, cols, cols, along, mode, block, int(rht), 3, 9, 2, ctypes.byref(ct),
+           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return st
+
+
+def _poll(nv):
+    p = nv.lib().nvfp4_poll_noalloc
+    p.argtypes = [ctypes.c_void_p]
+    p.restype = ctypes.c_int
+    return p(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_noalloc_empty_and_refused_shapes_match_workspace_entry_point():
+    # zero rows: status 0 and a tensor scale of 1, as nvfp4_quantize gives; a shape that
+    # nvfp4_quantize refuses before any device work is refused with the same status
+    nv, f = _entry()
+    out = nv.NVFP4Tensor.empty(16, 64, 0)
+    out.tensor_scale.fill_(7.0)
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    assert _call(nv, f, x, 0, 64, 0, 0, 0, False, out) == 0
+    torch.cuda.synchronize()
+    assert out.tensor_scale.item() == 1.0
+    ws = nv.Workspace()
+    x = torch.ones((24, 64), dtype=torch.bfloat16, device="cuda")    # along = 1 needs rows % 16 == 0
+    ref_st = nv.lib().nvfp4_quantize(ctypes.c_void_p(x.data_ptr()), 24, 64, 64, 1, 0, 0, 0, 3, 9, 2,
+                                     ctypes.byref(nv.NVFP4Tensor.empty(64, 24, 0).c()), ws.ptr, None)
+    assert ref_st == 3
+    assert _call(nv, f, x, 24, 64, 1, 0, 0, False, nv.NVFP4Tensor.empty(64, 24, 0)) == ref_st
+
+
+def test_noalloc_poll_reports_and_clears_device_flags():
+    # a non-finite input is flagged in the library's array and reported once by the poll
+    nv, f = _entry()
+    assert _poll(nv) == 0
+    x = torch.ones((32, 32), dtype=torch.bfloat16, device="cuda")
+    x[3, 5] = float("nan")
+    assert _call(nv, f, x, 32, 32, 0, 0, 0, False, nv.NVFP4Tensor.empty(32, 32, 0)) == 0
+    assert _poll(nv) == 7
+    assert _poll(nv) == 0
+    x[3, 5] = 1.0
+    assert _call(nv, f, x, 32, 32, 0, 0, 0, False, nv.NVFP4Tensor.empty(32, 32, 0)) == 0
+    assert _poll(nv) == 0
