@@ -125,10 +125,12 @@ class ClockSampler:
                 "samples": len(rows), "samples_under_load": len(loaded), "sm_mhz_min": min(sm)}
 
 
-def linear_config() -> dict:
+def linear_config(world: int = 1) -> dict:
     """The workload of the default line (both arms report it)."""
     return {"workload": "NVFP4 linear fwd+bwd: fprop 8192x20480x5120, dgrad 8192x5120x20480, "
                         "wgrad 20480x5120x8192, W 16x16 quantized every step",
+            "parallelism": f"dp{world}" + (" (amax all-reduce between quantize passes, dW reduce-scatter "
+                                           "overlapping dgrad)" if world > 1 else ""),
             "tokens": T_TOK, "d_in": D_IN, "d_out": D_OUT, "rht": "16-point, wgrad operands",
             "sr": "Philox4x32-10, dY both forms",
             "l2": "256 MiB buffer written between timed steps (outside the events); inputs 629 MB > L2"}
@@ -175,10 +177,20 @@ def run_ours(args, rank, world, local_rank):
     dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
-    # The step as a user runs it: the two public entry points of the linear layer.
+    # The step as a user runs it: the two public entry points of the linear layer.  Over N > 1
+    # ranks each rank holds its own 8192 tokens of an N x 8192-token batch and the step is the
+    # data-parallel one: the amax of X and dY all-reduced between the quantize passes (every
+    # rank's forms are its slice of the whole batch's), and the dW partial sums reduce-scattered
+    # over NCCL while the dgrad GEMM runs.
+    dp = nv.DPLinear(T_TOK, D_IN, D_OUT, rht_seed=0, device=dev) if world > 1 else None
+
     def step(sr_seed):
-        nv.nvfp4_linear_fwd(ctx, x, w, y)
-        nv.nvfp4_linear_bwd(ctx, dy, sr_seed, dx, dw)
+        if dp is None:
+            nv.nvfp4_linear_fwd(ctx, x, w, y)
+            nv.nvfp4_linear_bwd(ctx, dy, sr_seed, dx, dw)
+        else:
+            dp.fwd(x, w, y)
+            dp.bwd(dy, sr_seed, dx)
 
     # The same step as the sequence of public calls that nvfp4_linear_fwd / nvfp4_linear_bwd
     # make, with an event between calls: the per-kernel fields (roofline, quantize, per-GEMM).
@@ -252,7 +264,8 @@ def run_ours(args, rank, world, local_rank):
         hx, hw, hdy = (t.pin_memory() for t in (x_h, w_h, dy_h))
         hy = torch.empty((T_TOK, D_OUT), dtype=torch.bfloat16).pin_memory()
         hdx = torch.empty((T_TOK, D_IN), dtype=torch.bfloat16).pin_memory()
-        hdw = torch.empty((D_OUT, D_IN), dtype=torch.float32).pin_memory()
+        dw_dev = dw if dp is None else dp.dw          # over N > 1 ranks: this rank's rows of the batch's dW
+        hdw = torch.empty(tuple(dw_dev.shape), dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
         d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
 
@@ -280,13 +293,19 @@ def run_ours(args, rank, world, local_rank):
             comp.wait_event(xw_in)
             if prev["y_read"] is not None:
                 comp.wait_event(prev["y_read"])
-            nv.nvfp4_linear_fwd(ctx, x, w, y)
+            if dp is None:
+                nv.nvfp4_linear_fwd(ctx, x, w, y)
+            else:
+                dp.fwd(x, w, y)
             y_done = evt()
             y_done.record(comp)
             comp.wait_event(dy_in)
             if prev["dxdw_read"] is not None:
                 comp.wait_event(prev["dxdw_read"])
-            nv.nvfp4_linear_bwd(ctx, dy, seed, dx, dw)
+            if dp is None:
+                nv.nvfp4_linear_bwd(ctx, dy, seed, dx, dw)
+            else:
+                dp.bwd(dy, seed, dx)
             bwd_done = evt()
             bwd_done.record(comp)
             with torch.cuda.stream(down_s):
@@ -296,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
                 y_read.record(down_s)
                 down_s.wait_event(bwd_done)
                 hdx.copy_(dx, non_blocking=True)
-                hdw.copy_(dw, non_blocking=True)
+                hdw.copy_(dw_dev, non_blocking=True)
                 dxdw_read = evt()
                 dxdw_read.record(down_s)
             prev.update(bwd=bwd_done, y_read=y_read, dxdw_read=dxdw_read)
@@ -315,13 +334,14 @@ def run_ours(args, rank, world, local_rank):
         e1.record(comp)
         torch.cuda.synchronize()
         # the read-backs hold the last step's results
-        if not (torch.equal(hy, y.cpu()) and torch.equal(hdx, dx.cpu()) and torch.equal(hdw, dw.cpu())):
+        if not (torch.equal(hy, y.cpu()) and torch.equal(hdx, dx.cpu()) and torch.equal(hdw, dw_dev.cpu())):
             raise RuntimeError("end-to-end read-back differs from the device results")
         e2e_ms = reduce_max(e0.elapsed_time(e1), dist, dev) / args.e2e_steps
         e2e = {"value": job_tflops(world, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd -> pinned host Y, dX, dW; uploads, "
-                       "compute and read-backs on three event-ordered streams"}
+               "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd (N > 1: the data-parallel step) -> pinned "
+                       "host Y, dX, dW (N > 1: this rank's rows); uploads, compute and read-backs on three "
+                       "event-ordered streams"}
 
     ffn = ffn_fields(args, world, dev, dist, flush) if args.ffn else None
     if rank != 0:
@@ -341,7 +361,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 scale) operands, fp32 accumulate",
         "data": "synthetic (seeded N(0,1) X with 0.1% x50 outlier channels, N(0,0.02) W, N(0,1e-4) dY; bf16)",
-        "config": linear_config(),
+        "config": linear_config(world),
         "roofline": {"bound": "tensor", "kernel": "gemm_nvf4_2sm_kernel", "achieved": achieved,
                      "peak": peak_tensor, "unit": "TFLOP/s", "frac": achieved / peak_tensor,
                      "traffic": gemm_traffic(),

@@ -259,6 +259,67 @@ nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, i
  * device left in the library's array, with the precedence of nvfp4_poll.  Allocates nothing. */
 nvfp4_status nvfp4_poll_noalloc(nvfp4_stream_t stream);
 
+/*
+ * MXFP4, the format the pages compare NVFP4 against (gist.science 2.A: blocks of 32 elements with
+ * a power-of-two UE8M0 scale and no tensor scale; 4 "Ergebnisse": MXFP4 needs about 36 % more
+ * training tokens to match NVFP4).  One form per call, a single pass (no tensor amax):
+ *   scale code of a block = floor(log2 amax_b) - 2 + 127 clamped to [0, 254] (0 for an all-zero
+ *   block), i.e. 2^E with E the block's exponent less that of E2M1's largest value (6 = 1.5 * 2^2);
+ *   element u = v * 2^-E, encoded to E2M1 as in nvfp4_quantize (RNE, or SR with the same Philox
+ *   fields indexed by the element's position in the form).
+ * Layout: codes [rows][k/2] as for NVFP4; scales in 128x4 tiles of 512 bytes, entry (r, kb =
+ * k_index/32) at ((r/128)*ceil(k/128) + kb/4)*512 + (r%32)*16 + ((r/32)%4)*4 + kb%4 (zero padding),
+ * the layout the tcgen05 kind::mxf4 MMA reads.
+ * Shape rules: k % 32 == 0 (k = cols for along = 0, rows for along = 1); along = 1 needs
+ * rows % 32 == 0; cols % 16 == 0.  Non-finite inputs are out of contract (not flagged).  ws
+ * receives the timeout flag of the tile copies.
+ */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    int64_t rows;
+    int64_t k;
+} nvfp4_mx_tensor;
+
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k); /* ceil(rows/128)*128 * ceil(k/128)*4 */
+nvfp4_status nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along,
+                               nvfp4_round mode, uint64_t sr_seed, uint32_t stream_id,
+                               nvfp4_mx_tensor* out, void* ws, nvfp4_stream_t stream);
+/* D[M][N] = sum_k A[m][k] * B[n][k] over MXFP4 forms with the same k, by the tcgen05
+ * kind::mxf4 block-scaled MMA; fp32 accumulation, bf16 or fp32 output.  Shape rules and kernel
+ * choice as nvfp4_gemm (K % 32 == 0). */
+nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor* a, const nvfp4_mx_tensor* b, void* d, int64_t ldd,
+                           nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream);
+
+/*
+ * BF16 path for the linear layers the recipe keeps in high precision (gist.science 2.B.1: about
+ * 15 % of the linear layers, mostly the last ones, stay in BF16).  The GEMM is the same SM-pair
+ * tcgen05 kernel as nvfp4_gemm with kind::f16 MMAs (bf16 operands, fp32 accumulation in TMEM).
+ *
+ * nvfp4_bf16_gemm: D[M][N] = A[M][K] . B[N][K]^T, A and B bf16 row-major (K-major) with leading
+ * dimensions lda, ldb (elements); bf16 or fp32 output.  Shape rules: M, N >= 1; K >= 8, K % 8 == 0;
+ * lda >= K, ldb >= K, both % 8 == 0; ldd >= N, ldd * sizeof(out) % 16 == 0.  ws: timeout flag.
+ */
+nvfp4_status nvfp4_bf16_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, int64_t M, int64_t N,
+                             int64_t K, void* d, int64_t ldd, nvfp4_dtype out_dtype, void* ws,
+                             nvfp4_stream_t stream);
+/* xt[c][r] = x[r][c] for bf16 x[rows][ldx] into xt[cols][ldxt]; rows % 8 == 0, cols % 8 == 0,
+ * ldx and ldxt multiples of 8 (elements). */
+nvfp4_status nvfp4_bf16_transpose(const void* x, int64_t rows, int64_t cols, int64_t ldx, void* xt,
+                                  int64_t ldxt, nvfp4_stream_t stream);
+/* The BF16 linear layer y = x w^T (x [T][d], w [n][d], dy [T][n], all bf16 contiguous):
+ *   fwd: y [T][n] (bf16) = x . w^T;
+ *   bwd: dx [T][d] (bf16) = dy . w and dw [n][d] (fp32) = dy^T . x, through the K-major
+ *        transposes w^T, dy^T and x^T written into `scratch` (caller-owned,
+ *        nvfp4_linear_bf16_scratch_bytes(T, d, n) bytes, 16-byte aligned).  dx or dw may be NULL.
+ * Shape rules: T, d, n positive multiples of 8. */
+size_t nvfp4_linear_bf16_scratch_bytes(int64_t T, int64_t d, int64_t n);
+nvfp4_status nvfp4_linear_bf16_fwd(const void* x, const void* w, void* y, int64_t T, int64_t d, int64_t n,
+                                   void* ws, nvfp4_stream_t stream);
+nvfp4_status nvfp4_linear_bf16_bwd(const void* x, const void* w, const void* dy, void* dx, float* dw,
+                                   int64_t T, int64_t d, int64_t n, void* scratch, void* ws,
+                                   nvfp4_stream_t stream);
+
 /* Synchronize `stream`, then report (and clear) the device flags of `ws`: NVFP4_ERR_TIMEOUT
  * takes precedence over NVFP4_ERR_NONFINITE; NVFP4_OK when neither is set. */
 nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream);

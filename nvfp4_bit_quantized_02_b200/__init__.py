@@ -44,6 +44,10 @@ class CTensor(ctypes.Structure):
                 ("block", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class CMXTensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64), ("k", ctypes.c_int64)]
+
+
 class CLinearCtx(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("n", ctypes.c_int64), ("rht_seed", ctypes.c_uint64),
                 ("xq", CTensor), ("xq_rht", CTensor), ("wq", CTensor), ("wqt", CTensor), ("dyq", CTensor),
@@ -84,6 +88,14 @@ def _lib():
             "nvfp4_gelu_fwd_amax": ([vp, vp, i64, i64, u64, vp, vp], i32),
             "nvfp4_gelu_bwd_amax": ([vp, vp, vp, i64, i64, u64, vp, vp], i32),
             "nvfp4_poll": ([vp, vp], i32),
+            "nvfp4_mx_scales_bytes": ([i64, i64], c.c_size_t),
+            "nvfp4_bf16_gemm": ([vp, i64, vp, i64, i64, i64, i64, vp, i64, i32, vp, vp], i32),
+            "nvfp4_bf16_transpose": ([vp, i64, i64, i64, vp, i64, vp], i32),
+            "nvfp4_linear_bf16_scratch_bytes": ([i64, i64, i64], c.c_size_t),
+            "nvfp4_linear_bf16_fwd": ([vp, vp, vp, i64, i64, i64, vp, vp], i32),
+            "nvfp4_linear_bf16_bwd": ([vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
+            "nvfp4_mx_quantize": ([vp, i64, i64, i64, i32, i32, u64, u32, c.POINTER(CMXTensor), vp, vp], i32),
+            "nvfp4_mx_gemm": ([c.POINTER(CMXTensor), c.POINTER(CMXTensor), vp, i64, i32, vp, vp], i32),
             "nvfp4_quantize_noalloc": ([vp, i64, i64, i64, i32, i32, i32, i32, u64, u64, u32, T, vp], i32),
             "nvfp4_poll_noalloc": ([vp], i32),
             "nvfp4_set_wait_budget_ns": ([u64], None),
@@ -349,6 +361,108 @@ def nvfp4_gelu_bwd_amax(h: torch.Tensor, dg: torch.Tensor, out: torch.Tensor | N
 
 
 # ---------------------------------------------------------------------------------------
+# MXFP4 (the comparison format: blocks of 32, UE8M0 scales, no tensor scale)
+# ---------------------------------------------------------------------------------------
+@dataclass
+class MXTensor:
+    """One MXFP4 operand form (device buffers owned by torch)."""
+    codes: torch.Tensor          # uint8 [rows][k/2]
+    scales: torch.Tensor         # uint8, 128x4-tile swizzled UE8M0 block scales
+    rows: int
+    k: int
+
+    @staticmethod
+    def empty(rows: int, k: int, device=None) -> "MXTensor":
+        L = _lib()
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        codes = torch.empty(max(L.nvfp4_codes_bytes(rows, k), 1), dtype=torch.uint8, device=device)
+        scales = torch.empty(max(L.nvfp4_mx_scales_bytes(rows, k), 16), dtype=torch.uint8, device=device)
+        return MXTensor(codes, scales, rows, k)
+
+    def c(self) -> CMXTensor:
+        return CMXTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
+
+
+def nvfp4_mx_quantize(x: torch.Tensor, along: int = 0, mode: int = RNE, sr_seed: int = 0, stream_id: int = 0,
+                      out: MXTensor | None = None, ws: Workspace | None = None, stream=None) -> MXTensor:
+    rows, cols, ld = _bf16_2d(x)
+    R, K = (cols, rows) if along else (rows, cols)
+    out = out or MXTensor.empty(R, K, x.device)
+    ws = ws or default_workspace()
+    ct = out.c()
+    _check(_lib().nvfp4_mx_quantize(_ptr(x), rows, cols, ld, along, mode, sr_seed, stream_id, ctypes.byref(ct), ws.ptr,
+                                    _stream(stream)), "nvfp4_mx_quantize")
+    return out
+
+
+def nvfp4_mx_gemm(a: MXTensor, b: MXTensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                  ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D[M][N] = A . B^T over MXFP4 forms (kind::mxf4 block-scaled MMA)."""
+    if out is None:
+        out = torch.empty((a.rows, b.rows), dtype=out_dtype, device=a.codes.device)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("output must be bf16 or fp32")
+    code = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
+    ws = ws or default_workspace()
+    ca, cb = a.c(), b.c()
+    _check(_lib().nvfp4_mx_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), out.stride(0), code, ws.ptr,
+                                _stream(stream)), "nvfp4_mx_gemm")
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# BF16 path (the layers kept in high precision)
+# ---------------------------------------------------------------------------------------
+def nvfp4_bf16_gemm(a: torch.Tensor, b: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                    ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D[M][N] = A[M][K] . B[N][K]^T for bf16 A, B (tcgen05 kind::f16, fp32 accumulation)."""
+    M, K, lda = _bf16_2d(a)
+    N, Kb, ldb = _bf16_2d(b)
+    if Kb != K:
+        raise ValueError("A and B need the same K")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    code = OUT_FP32 if out.dtype == torch.float32 else OUT_BF16
+    ws = ws or default_workspace()
+    _check(_lib().nvfp4_bf16_gemm(_ptr(a), lda, _ptr(b), ldb, M, N, K, _ptr(out), out.stride(0), code, ws.ptr,
+                                  _stream(stream)), "nvfp4_bf16_gemm")
+    return out
+
+
+def nvfp4_bf16_transpose(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    rows, cols, ld = _bf16_2d(x)
+    out = torch.empty((cols, rows), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(_lib().nvfp4_bf16_transpose(_ptr(x), rows, cols, ld, _ptr(out), out.stride(0), _stream(stream)),
+           "nvfp4_bf16_transpose")
+    return out
+
+
+class LinearBF16:
+    """The BF16 linear layer y = x w^T with its caller-owned transpose scratch."""
+
+    def __init__(self, T: int, d: int, n: int, device=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.T, self.d, self.n = T, d, n
+        self.scratch = torch.empty(max(_lib().nvfp4_linear_bf16_scratch_bytes(T, d, n), 16), dtype=torch.uint8,
+                                   device=device)
+        self.ws = Workspace(device)
+
+    def fwd(self, x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        y = torch.empty((self.T, self.n), dtype=torch.bfloat16, device=x.device) if y is None else y
+        _check(_lib().nvfp4_linear_bf16_fwd(_ptr(x), _ptr(w), _ptr(y), self.T, self.d, self.n, self.ws.ptr,
+                                            _stream(stream)), "nvfp4_linear_bf16_fwd")
+        return y
+
+    def bwd(self, x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor, dx: torch.Tensor | None = None,
+            dw: torch.Tensor | None = None, stream=None):
+        dx = torch.empty((self.T, self.d), dtype=torch.bfloat16, device=x.device) if dx is None else dx
+        dw = torch.empty((self.n, self.d), dtype=torch.float32, device=x.device) if dw is None else dw
+        _check(_lib().nvfp4_linear_bf16_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), self.T, self.d, self.n,
+                                            _ptr(self.scratch), self.ws.ptr, _stream(stream)), "nvfp4_linear_bf16_bwd")
+        return dx, dw
+
+
+# ---------------------------------------------------------------------------------------
 # linear layer
 # ---------------------------------------------------------------------------------------
 class LinearContext:
@@ -384,6 +498,78 @@ class LinearContext:
     @amax_ready.setter
     def amax_ready(self, v: bool):
         self.ctx.amax_ready = 1 if v else 0
+
+
+# ---------------------------------------------------------------------------------------
+# data parallelism over tokens
+# ---------------------------------------------------------------------------------------
+def dp_token_rows(T_local: int, rank: int, world: int):
+    """(row_offset, rows_total) of this rank's token shard in the whole batch: ranks hold equal
+    consecutive shards in rank order."""
+    return rank * T_local, world * T_local
+
+
+def dp_dw_rows(n: int, rank: int, world: int):
+    """The rows [r0, r1) of dW that the reduce-scatter leaves on this rank (n % world == 0)."""
+    if n % world:
+        raise ValueError("out-features must divide evenly over the ranks")
+    per = n // world
+    return rank * per, (rank + 1) * per
+
+
+class DPLinear:
+    """The NVFP4 linear layer y = x w^T under data parallelism: each rank holds T consecutive tokens
+    of a world * T-token batch and a replica of w.
+
+    - X and dY: the tensor scale comes from the whole batch, so the plain and RHT amax of each
+      rank's shard are all-reduced with an integer MAX between the two quantize passes, and SR
+      fields are indexed in the whole batch's forms: every rank's forms are its slice of the forms
+      one GPU would compute for the whole batch.
+    - W: quantized on every rank from the same replica (identical forms, no exchange).
+    - dW: each rank's wgrad GEMM gives the partial sum over its tokens; the partials are
+      reduce-scattered (fp32 sum) over the group, each rank keeping rows dp_dw_rows(n, rank,
+      world).  The wgrad GEMM runs first and the reduce-scatter overlaps the dgrad GEMM.
+    """
+
+    def __init__(self, T: int, d: int, n: int, group=None, rht_seed: int = 0, device=None):
+        import torch.distributed as dist
+        self.group = group
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.T, self.d, self.n, self.rht_seed = T, d, n, rht_seed
+        self.ctx = LinearContext(T, d, n, rht_seed=rht_seed, device=device)
+        self.dw_partial = torch.empty((n, d), dtype=torch.float32, device=device)
+        r0, r1 = dp_dw_rows(n, self.rank, self.world)
+        self.dw = torch.empty((r1 - r0, d), dtype=torch.float32, device=device)
+
+    def fwd(self, x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        c = self.ctx
+        off, total = dp_token_rows(self.T, self.rank, self.world)
+        nvfp4_quantize_dual_dp(x, self.group, off, total, mode=RNE, rht_seed=self.rht_seed, out_row=c.xq,
+                               out_col=c.xq_rht, ws=c.ws)
+        nvfp4_quantize_weight(w, out=c.wq, out_t=c.wqt, ws=c.ws)
+        return nvfp4_gemm(c.xq, c.wq, out=y, ws=c.ws)
+
+    def bwd(self, dy: torch.Tensor, sr_seed: int, dx: torch.Tensor | None = None):
+        """dX for this rank's tokens; this rank's rows of the batch's dW land in self.dw."""
+        import torch.distributed as dist
+        c = self.ctx
+        off, total = dp_token_rows(self.T, self.rank, self.world)
+        nvfp4_quantize_dual_dp(dy, self.group, off, total, mode=SR, rht_seed=self.rht_seed, sr_seed=sr_seed,
+                               stream_row=STREAM_DGRAD, stream_col=STREAM_WGRAD, out_row=c.dyq, out_col=c.dyq_rht,
+                               ws=c.ws)
+        nvfp4_gemm(c.dyq_rht, c.xq_rht, out=self.dw_partial, ws=c.ws)
+        work = None
+        if self.world > 1:
+            work = dist.reduce_scatter_tensor(self.dw, self.dw_partial, op=dist.ReduceOp.SUM, group=self.group,
+                                              async_op=True)
+        dx = nvfp4_gemm(c.dyq, c.wqt, out=dx, ws=c.ws)
+        if work is not None:
+            work.wait()
+        else:
+            self.dw.copy_(self.dw_partial)
+        return dx
 
 
 def nvfp4_linear_fwd(ctx: LinearContext, x: torch.Tensor, w: torch.Tensor | None, y: torch.Tensor | None = None,

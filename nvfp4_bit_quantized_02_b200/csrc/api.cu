@@ -482,6 +482,122 @@ nvfp4_status nvfp4_gelu_bwd_amax(const void* h, const void* dg, void* dh, int64_
     return gelu_amax(true, h, dg, dh, rows, cols, rht_seed, ws, stream);
 }
 
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k) {
+    if (rows <= 0 || k <= 0) return 0;
+    return (size_t)(((rows + 127) / 128) * 128 * ((k + 127) / 128) * 4);
+}
+
+nvfp4_status nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along, nvfp4_round mode,
+                               uint64_t sr_seed, uint32_t stream_id, nvfp4_mx_tensor* out, void* ws,
+                               nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
+    if (along != 0 && along != 1) return NVFP4_ERR_ARG;
+    if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
+    if (!out || !out->codes || !out->scales) return NVFP4_ERR_NULL;
+    if (!aligned16(out->codes) || !aligned16(out->scales)) return NVFP4_ERR_ALIGN;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    const int64_t R = along ? cols : rows, K = along ? rows : cols;
+    if (K % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    out->rows = R;
+    out->k = K;
+    if (R == 0 || K == 0) return NVFP4_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((R & 127) != 0 || ((K >> 5) & 3) != 0)
+        if (cudaError_t e = cudaMemsetAsync(out->scales, 0, nvfp4_mx_scales_bytes(R, K), s)) return from_cuda(e);
+    MxParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = reinterpret_cast<const uint16_t*>(x);
+    p.rows = rows;
+    p.cols = cols;
+    p.ld = ldx;
+    p.codes = out->codes;
+    p.scales = out->scales;
+    p.nkt = (K + 127) / 128;
+    p.sr = mode == NVFP4_SR;
+    p.stream_id = stream_id;
+    p.flags = &ws_of(ws)->flags;
+    return from_cuda(launch_quantize_mx(p, along == 1, sr_seed, s));
+}
+
+nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor* a, const nvfp4_mx_tensor* b, void* d, int64_t ldd,
+                           nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream) {
+    if (!a || !b || !d || !a->codes || !a->scales || !b->codes || !b->scales) return NVFP4_ERR_NULL;
+    if (!aligned16(a->codes) || !aligned16(a->scales) || !aligned16(b->codes) || !aligned16(b->scales))
+        return NVFP4_ERR_ALIGN;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32) return NVFP4_ERR_ARG;
+    const int64_t M = a->rows, N = b->rows, K = a->k;
+    if (b->k != K) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return NVFP4_ERR_LIMIT;
+    const int64_t esz = out_dtype == NVFP4_OUT_FP32 ? 4 : 2;
+    if (ldd < N) return NVFP4_ERR_SHAPE;
+    if (!aligned16(d) || (ldd * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gemm_mxf4(a->codes, a->scales, M, b->codes, b->scales, N, K, d, ldd,
+                                      out_dtype == NVFP4_OUT_FP32, &ws_of(ws)->flags, g_budget_ns.load(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_bf16_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, int64_t M, int64_t N, int64_t K,
+                             void* d, int64_t ldd, nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream) {
+    if (!a || !b || !d) return NVFP4_ERR_NULL;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 1 || K < 8 || K % 8 != 0 || lda < K || ldb < K) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return NVFP4_ERR_LIMIT;
+    const int64_t esz = out_dtype == NVFP4_OUT_FP32 ? 4 : 2;
+    if (ldd < N) return NVFP4_ERR_SHAPE;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d) || lda % 8 || ldb % 8 || (ldd * esz) % 16) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gemm_bf16(reinterpret_cast<const uint16_t*>(a), lda, reinterpret_cast<const uint16_t*>(b), ldb,
+                                      M, N, K, d, ldd, out_dtype == NVFP4_OUT_FP32, &ws_of(ws)->flags, g_budget_ns.load(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_bf16_transpose(const void* x, int64_t rows, int64_t cols, int64_t ldx, void* xt, int64_t ldxt,
+                                  nvfp4_stream_t stream) {
+    if (rows < 0 || cols < 0 || rows % 8 || cols % 8 || ldx < cols || ldxt < rows) return NVFP4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NVFP4_OK;
+    if (!x || !xt) return NVFP4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(xt) || ldx % 8 || ldxt % 8) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_transpose_bf16(reinterpret_cast<const uint16_t*>(x), rows, cols, ldx,
+                                           reinterpret_cast<uint16_t*>(xt), ldxt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_linear_bf16_scratch_bytes(int64_t T, int64_t d, int64_t n) {
+    if (T <= 0 || d <= 0 || n <= 0) return 0;
+    return (size_t)(2 * (d * n + n * T + d * T));
+}
+
+nvfp4_status nvfp4_linear_bf16_fwd(const void* x, const void* w, void* y, int64_t T, int64_t d, int64_t n, void* ws,
+                                   nvfp4_stream_t stream) {
+    if (T <= 0 || d <= 0 || n <= 0 || T % 8 || d % 8 || n % 8) return NVFP4_ERR_SHAPE;
+    return nvfp4_bf16_gemm(x, d, w, d, T, n, d, y, n, NVFP4_OUT_BF16, ws, stream);
+}
+
+nvfp4_status nvfp4_linear_bf16_bwd(const void* x, const void* w, const void* dy, void* dx, float* dw, int64_t T,
+                                   int64_t d, int64_t n, void* scratch, void* ws, nvfp4_stream_t stream) {
+    if (T <= 0 || d <= 0 || n <= 0 || T % 8 || d % 8 || n % 8) return NVFP4_ERR_SHAPE;
+    if (!x || !w || !dy || !scratch) return NVFP4_ERR_NULL;
+    if (!aligned16(scratch)) return NVFP4_ERR_ALIGN;
+    uint16_t* wt = reinterpret_cast<uint16_t*>(scratch);   // [d][n]
+    uint16_t* dyt = wt + d * n;                             // [n][T]
+    uint16_t* xt = dyt + n * T;                             // [d][T]
+    if (dx) {
+        if (nvfp4_status st = nvfp4_bf16_transpose(w, n, d, d, wt, n, stream)) return st;
+        if (nvfp4_status st = nvfp4_bf16_gemm(dy, n, wt, n, T, d, n, dx, d, NVFP4_OUT_BF16, ws, stream)) return st;
+    }
+    if (dw) {
+        if (nvfp4_status st = nvfp4_bf16_transpose(dy, T, n, n, dyt, T, stream)) return st;
+        if (nvfp4_status st = nvfp4_bf16_transpose(x, T, d, d, xt, T, stream)) return st;
+        if (nvfp4_status st = nvfp4_bf16_gemm(dyt, T, xt, T, n, d, T, dw, d, NVFP4_OUT_FP32, ws, stream)) return st;
+    }
+    return NVFP4_OK;
+}
+
 nvfp4_status nvfp4_poll(void* ws, nvfp4_stream_t stream) {
     if (!ws) return NVFP4_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

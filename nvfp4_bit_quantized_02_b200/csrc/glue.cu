@@ -62,11 +62,17 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(const uint4* __restrict__
 
 // ---------------------------------------------------------------------------------------
 // GeLU forward or backward with the amax of its bf16 output fused in (the amax pass of the
-// next quantize, which reads this output, is then skipped): a thread takes a 16-row x 4-column
-// patch of the [rows][cols] output, writes it, and reduces its plain magnitudes (as packed
-// bf16 integers) and its 16-point RHT along rows (fp32), exactly as the amax pass does.
+// next quantize, which reads this output, is then skipped).  A CTA takes 16-row x 512-column
+// tiles of the [rows][cols] output:
+//   1. each thread computes four 16-byte chunks (8 elements of one row) with coalesced 16-byte
+//      loads and stores, reduces the plain magnitudes as packed bf16 integers, and stages the
+//      bf16 results in shared memory;
+//   2. each thread takes one column pair of the staged tile (16 rows x 2 columns, one 32-bit
+//      shared load per row), applies the 16-point RHT along the rows as f32x2 pairs and reduces
+//      the transformed magnitudes -- exactly what the amax pass computes from this output.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ uint2 ld_patch_row(const uint16_t* p) { return *reinterpret_cast<const uint2*>(p); }
+constexpr int kGaRows = 16, kGaCols = 512, kGaThreads = 256;
+constexpr int kGaChunks = kGaRows * kGaCols / 8;   // 1024 sixteen-byte chunks per tile
 
 __device__ __forceinline__ uint32_t warp_max_u32_g(uint32_t v) {
 #pragma unroll
@@ -88,53 +94,127 @@ __device__ __forceinline__ void block_max_to(uint32_t v, uint32_t* dst, uint32_t
 }
 
 template <bool BWD>
-__global__ void __launch_bounds__(256, 2) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
-                                                        uint16_t* __restrict__ out, int64_t rows, int64_t cols,
-                                                        uint32_t signs, uint32_t* __restrict__ amax_plain,
-                                                        uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
-    __shared__ uint32_t red[8];
-    const int64_t cpr = cols >> 2;
-    const int64_t total = (rows >> 4) * cpr;
+__device__ __forceinline__ uint4 gelu_chunk(const uint4 x, const uint4 d) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const uint32_t e[4] = {d.x, d.y, d.z, d.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        o[j] = BWD ? f32x2_to_bf16x2(bf16_lo(e[j]) * gelu_grad_f(bf16_lo(w[j])), bf16_hi(e[j]) * gelu_grad_f(bf16_hi(w[j])))
+                   : f32x2_to_bf16x2(gelu_f(bf16_lo(w[j])), gelu_f(bf16_hi(w[j])));
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(kGaThreads) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
+                                                            uint16_t* __restrict__ out, int64_t rows, int64_t cols,
+                                                            const SignMasks sm, uint32_t* __restrict__ amax_plain,
+                                                            uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
+    __shared__ __align__(16) uint16_t tile[kGaRows * kGaCols];
+    __shared__ uint32_t red[kGaThreads / 32];
+    const int tid = threadIdx.x;
+    const int64_t ntc = (cols + kGaCols - 1) / kGaCols;
+    const int64_t ntiles = (rows / kGaRows) * ntc;
     uint32_t m = 0;
     float mr = 0.0f;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t g = u / cpr, k = u - g * cpr;
-        const int64_t base = (g << 4) * cols + (k << 2);
-        uint2 v[16];
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t tr = t / ntc, tc = t - tr * ntc;
+        const int64_t r0 = tr * kGaRows, c0 = tc * kGaCols;
+        // 1. GeLU of four chunks per thread: loads first, then compute, store and stage
+        uint4 x[kGaChunks / kGaThreads], d[kGaChunks / kGaThreads];
+        bool ok[kGaChunks / kGaThreads];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint2 x = ld_patch_row(h + base + i * cols);
-            if (BWD) {
-                const uint2 d = ld_patch_row(dg + base + i * cols);
-                v[i].x = f32x2_to_bf16x2(bf16_lo(d.x) * gelu_grad_f(bf16_lo(x.x)), bf16_hi(d.x) * gelu_grad_f(bf16_hi(x.x)));
-                v[i].y = f32x2_to_bf16x2(bf16_lo(d.y) * gelu_grad_f(bf16_lo(x.y)), bf16_hi(d.y) * gelu_grad_f(bf16_hi(x.y)));
-            } else {
-                v[i].x = f32x2_to_bf16x2(gelu_f(bf16_lo(x.x)), gelu_f(bf16_hi(x.x)));
-                v[i].y = f32x2_to_bf16x2(gelu_f(bf16_lo(x.y)), gelu_f(bf16_hi(x.y)));
-            }
-            *reinterpret_cast<uint2*>(out + base + i * cols) = v[i];
-            m = __vmaxu2(m, v[i].x & 0x7FFF7FFFu);
-            m = __vmaxu2(m, v[i].y & 0x7FFF7FFFu);
+        for (int u = 0; u < kGaChunks / kGaThreads; ++u) {
+            const int j = tid + u * kGaThreads, i = j / (kGaCols / 8), ch = j % (kGaCols / 8);
+            const int64_t col = c0 + ch * 8;
+            ok[u] = col < cols;
+            const int64_t off = (r0 + i) * cols + col;
+            x[u] = ok[u] ? *reinterpret_cast<const uint4*>(h + off) : make_uint4(0, 0, 0, 0);
+            d[u] = (BWD && ok[u]) ? *reinterpret_cast<const uint4*>(dg + off) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            float a[16], b[16];
+        for (int u = 0; u < kGaChunks / kGaThreads; ++u) {
+            const int j = tid + u * kGaThreads, i = j / (kGaCols / 8), ch = j % (kGaCols / 8);
+            const uint4 o = ok[u] ? gelu_chunk<BWD>(x[u], d[u]) : make_uint4(0, 0, 0, 0);
+            if (ok[u]) *reinterpret_cast<uint4*>(out + (r0 + i) * cols + c0 + ch * 8) = o;
+            *reinterpret_cast<uint4*>(tile + i * kGaCols + ch * 8) = o;
+            m = __vmaxu2(m, o.x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, o.y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, o.z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, o.w & 0x7FFF7FFFu);
+        }
+        __syncthreads();
+        // 2. the RHT amax of one column pair per thread (zero columns past `cols` add nothing)
+        {
+            uint64_t f[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                f[i] = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(tile + i * kGaCols + 2 * tid) ^ sm.m[i]);
+            rht16_pairs(f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t w = p == 0 ? v[i].x : v[i].y;
-                a[i] = bf16_lo(w);
-                b[i] = bf16_hi(w);
+                float a, b;
+                f2_split(f[i], a, b);
+                mr = max3_abs(mr, a, b);
             }
-            rht16(a, signs);
-            rht16(b, signs);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) mr = fmaxf(mr, fmaxf(fabsf(a[i]), fabsf(b[i])));
         }
+        __syncthreads();
     }
     const uint32_t mag = max(m & 0xFFFFu, m >> 16);
     if (mag >= 0x7F80u || !(mr < __int_as_float(0x7F800000))) atomicOr(flags, kFlagNonFinite);
     block_max_to(mag << 16, amax_plain, red);
     block_max_to(__float_as_uint(mr), amax_rht, red);
+}
+
+// ---------------------------------------------------------------------------------------
+// bf16 transpose xt[c][r] = x[r][c] (the K-major operands of the BF16 path's dgrad and wgrad):
+// 64 x 64 tiles through shared memory, 16-byte loads and stores on both sides; rows % 8 == 0,
+// cols % 8 == 0.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                                                             int64_t ldx, uint16_t* __restrict__ xt, int64_t ldt) {
+    __shared__ uint16_t t[64][64 + 2];
+    const int tid = threadIdx.x;
+    const int64_t ntc = (cols + 63) / 64, ntiles = ((rows + 63) / 64) * ntc;
+    for (int64_t it = blockIdx.x; it < ntiles; it += gridDim.x) {
+        const int64_t r0 = (it / ntc) * 64, c0 = (it % ntc) * 64;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = tid + 256 * u, r = j >> 3, ch = j & 7;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r0 + r < rows && c0 + ch * 8 < cols) v = *reinterpret_cast<const uint4*>(x + (r0 + r) * ldx + c0 + ch * 8);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                t[r][ch * 8 + 2 * e] = (uint16_t)(w[e] & 0xFFFFu);
+                t[r][ch * 8 + 2 * e + 1] = (uint16_t)(w[e] >> 16);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = tid + 256 * u, c = j >> 3, ch = j & 7;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w[e] = (uint32_t)t[ch * 8 + 2 * e][c] | ((uint32_t)t[ch * 8 + 2 * e + 1][c] << 16);
+            if (c0 + c < cols && r0 + ch * 8 < rows)
+                *reinterpret_cast<uint4*>(xt + (c0 + c) * ldt + r0 + ch * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, uint16_t* xt, int64_t ldt,
+                                  cudaStream_t s) {
+    const int64_t tiles = ((rows + 63) / 64) * ((cols + 63) / 64);
+    if (tiles == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * 8;
+    transpose_bf16_kernel<<<(int)(tiles < cap ? tiles : cap), 256, 0, s>>>(x, rows, cols, ldx, xt, ldt);
+    return cudaGetLastError();
 }
 
 static int elementwise_grid(int64_t n8) {
@@ -169,17 +249,19 @@ cudaError_t launch_gelu_bwd(const uint16_t* h, const uint16_t* dg, uint16_t* dh,
 cudaError_t launch_gelu_amax(bool bwd, const uint16_t* h, const uint16_t* dg, uint16_t* out, int64_t rows,
                              int64_t cols, uint32_t signs, uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags,
                              cudaStream_t s) {
-    const int64_t units = (rows >> 4) * (cols >> 2);
-    if (units == 0) return cudaSuccess;
+    const int64_t tiles = (rows / kGaRows) * ((cols + kGaCols - 1) / kGaCols);
+    if (tiles == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t want = (units + 255) / 256, cap = (int64_t)sms * 4;
-    const int grid = (int)(want < cap ? want : cap);
+    const int64_t cap = (int64_t)sms * 3;   // resident CTAs (16 KB of shared memory, <= 80 registers each)
+    const int grid = (int)(tiles < cap ? tiles : cap);
     if (bwd)
-        gelu_amax_kernel<true><<<grid, 256, 0, s>>>(h, dg, out, rows, cols, signs, amax_plain, amax_rht, flags);
+        gelu_amax_kernel<true><<<grid, kGaThreads, 0, s>>>(h, dg, out, rows, cols, sign_masks(signs), amax_plain, amax_rht,
+                                                           flags);
     else
-        gelu_amax_kernel<false><<<grid, 256, 0, s>>>(h, nullptr, out, rows, cols, signs, amax_plain, amax_rht, flags);
+        gelu_amax_kernel<false><<<grid, kGaThreads, 0, s>>>(h, nullptr, out, rows, cols, sign_masks(signs), amax_plain,
+                                                            amax_rht, flags);
     return cudaGetLastError();
 }
 

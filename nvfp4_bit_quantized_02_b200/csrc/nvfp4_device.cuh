@@ -28,6 +28,45 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Packed fp32 pairs: sm_100's f32x2 arithmetic performs two independent IEEE round-to-nearest
+// operations per instruction, bit-identical to two scalar __fadd_rn / __fsub_rn / __fmul_rn.
+// A pair is a 64-bit register {lo, hi}.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// the bf16 pair of a 32-bit word (low half = first element) widened to an fp32 pair (exact)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+    return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// max(a, |b|, |c|) in one instruction (three-input max of sm_100)
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
+// ---------------------------------------------------------------------------------------
 // E2M1 encode, round-to-nearest-even, saturating to +-6, sign kept.  Two values per
 // instruction; `lo` lands in bits [0,4), `hi` in bits [4,8).
 // ---------------------------------------------------------------------------------------
@@ -73,6 +112,29 @@ __device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
     const uint32_t lo = (cb + (65535u - 0x4B000000u) - r16) >> 16;
     const uint32_t code = a >= 0x3F800000u ? hi : lo;
     return ((b >> 28) & 8u) | code;
+}
+
+// The same decision for a pair of values (lo, hi) with their own 16-bit random fields; the
+// round-up add of the |u| < 1 branch is one f32x2 instruction.  Returns lo's code in bits [0,4)
+// and hi's in bits [4,8).
+__device__ __forceinline__ uint32_t e2m1_sr_pair(uint64_t u, uint32_t r_lo, uint32_t r_hi) {
+    float ul, uh;
+    f2_split(u, ul, uh);
+    const float afl = fminf(fabsf(ul), 6.0f), afh = fminf(fabsf(uh), 6.0f);
+    uint64_t cb2;
+    asm("fma.rp.f32x2 %0, %1, %2, %3;"
+        : "=l"(cb2)
+        : "l"(f2(afl, afh)), "l"(f2(131072.0f, 131072.0f)), "l"(f2(8388608.0f, 8388608.0f)));
+    float cbl, cbh;
+    f2_split(cb2, cbl, cbh);
+    const uint32_t al = __float_as_uint(afl), ah = __float_as_uint(afh);
+    const uint32_t hil = (al + (0x3FFFFFu - (252u << 22)) - (r_lo << 6)) >> 22;
+    const uint32_t hih = (ah + (0x3FFFFFu - (252u << 22)) - (r_hi << 6)) >> 22;
+    const uint32_t lol = (__float_as_uint(cbl) + (65535u - 0x4B000000u) - r_lo) >> 16;
+    const uint32_t loh = (__float_as_uint(cbh) + (65535u - 0x4B000000u) - r_hi) >> 16;
+    const uint32_t cl = (al >= 0x3F800000u ? hil : lol) | ((__float_as_uint(ul) >> 28) & 8u);
+    const uint32_t ch = (ah >= 0x3F800000u ? hih : loh) | ((__float_as_uint(uh) >> 28) & 8u);
+    return cl | (ch << 4);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -201,6 +263,24 @@ __device__ __forceinline__ void rht16(float (&v)[16], uint32_t signs) {
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+}
+
+// The same transform on two independent 16-vectors at once (the lo and hi halves of each pair),
+// with the signs already applied: each stage's adds and subtracts are f32x2 instructions.
+__device__ __forceinline__ void rht16_pairs(uint64_t (&v)[16]) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            const uint64_t a = v[i], b = v[i + h];
+            v[i] = f2_add(a, b);
+            v[i + h] = f2_sub(a, b);
+        }
+    }
+    const uint64_t q = f2(0.25f, 0.25f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = f2_mul(v[j], q);
 }
 
 // ---------------------------------------------------------------------------------------

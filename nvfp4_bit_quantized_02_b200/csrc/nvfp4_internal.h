@@ -19,6 +19,16 @@ static_assert(sizeof(Workspace) == 256, "workspace is 256 bytes");
 constexpr uint32_t kFlagNonFinite = 1u;
 constexpr uint32_t kFlagTimeout = 2u;
 
+// the 16 RHT signs as bf16-pair masks (0x80008000 for a -1 sign), a by-value kernel parameter
+struct SignMasks {
+    uint32_t m[16];
+};
+inline SignMasks sign_masks(uint32_t signs) {
+    SignMasks s;
+    for (int j = 0; j < 16; ++j) s.m[j] = ((signs >> j) & 1u) ? 0x80008000u : 0u;
+    return s;
+}
+
 // parameters of the tile quantizer (one read of x, up to two forms)
 struct QuantParams {
     const uint16_t* x;
@@ -46,11 +56,31 @@ struct QuantParams {
     uint32_t signs;
     uint64_t sr_seed;
     uint32_t* flags;  // workspace flags (timeout of a tile copy)
+    // filled by launch_quantize_tiles (constant-bank operands in the kernel):
+    uint32_t sign_mask2[16];  // RHT sign j as a bf16-pair mask: 0x80008000 when sign j is -1, else 0
+    uint32_t key0[10];        // Philox4x32-10 round keys of sr_seed (Weyl sequence of its two words)
+    uint32_t key1[10];
     // SR bit indexing of a token shard: x holds rows [row_offset, row_offset + rows) of a
     // rows_total-row tensor, and SR fields are indexed in the forms of that whole tensor
     int64_t row_offset;
     int64_t rows_total;
 };
+
+// parameters of the MXFP4 tile quantizer (one form per call)
+struct MxParams {
+    const uint16_t* x;
+    int64_t rows, cols, ld;    // the bf16 source [rows][ld]
+    uint8_t* codes;            // the form's codes [R][K/2]
+    uint8_t* scales;           // UE8M0 scales in 128x4 tiles
+    int64_t nkt;               // ceil(K / 128): 128x4 scale tiles per 128 form rows
+    int32_t sr;                // 1: stochastic rounding
+    uint32_t stream_id;
+    uint32_t* flags;           // workspace flags (timeout of a tile copy)
+    uint32_t key0[10];         // Philox4x32-10 round keys of the SR seed
+    uint32_t key1[10];
+};
+
+cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_seed, cudaStream_t s);
 
 cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax,
                               uint32_t* flags, cudaStream_t s);
@@ -64,6 +94,14 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
                              const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                              void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
                              cudaStream_t stream);
+cudaError_t launch_gemm_mxf4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M, const uint8_t* b_codes,
+                             const uint8_t* b_scales, int64_t N, int64_t K, void* d, int64_t ldd, bool out_fp32,
+                             uint32_t* flags, uint64_t budget_ns, cudaStream_t stream);
+cudaError_t launch_gemm_bf16(const uint16_t* a, int64_t lda, const uint16_t* b, int64_t ldb, int64_t M, int64_t N,
+                             int64_t K, void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
+                             cudaStream_t stream);
+cudaError_t launch_transpose_bf16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, uint16_t* xt, int64_t ldt,
+                                  cudaStream_t s);
 cudaError_t launch_gelu_fwd(const uint16_t* h, uint16_t* g, int64_t n, cudaStream_t s);
 cudaError_t launch_gelu_bwd(const uint16_t* h, const uint16_t* dg, uint16_t* dh, int64_t n, cudaStream_t s);
 cudaError_t launch_gelu_amax(bool bwd, const uint16_t* h, const uint16_t* dg, uint16_t* out, int64_t rows,

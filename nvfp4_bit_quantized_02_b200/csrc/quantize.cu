@@ -66,6 +66,28 @@ __device__ __forceinline__ void block_atomic_max(uint32_t v, uint32_t* dst, uint
     __syncthreads();
 }
 
+// A grid-stride walk over the (row, chunk) grid of a [rows][chunks_per_row] tensor without a
+// division per step: the stride S = gridDim * blockDim is split once into whole rows and a
+// remainder, and the position advances by carry.
+struct GridWalk {
+    int64_t r, k;            // current (row, chunk)
+    int64_t dr, dk, cpr;     // stride in rows and chunks, chunks per row
+    __device__ __forceinline__ GridWalk(int64_t start, int64_t stride, int64_t cpr_) : cpr(cpr_) {
+        r = start / cpr;
+        k = start - r * cpr;
+        dr = stride / cpr;
+        dk = stride - dr * cpr;
+    }
+    __device__ __forceinline__ void next() {
+        r += dr;
+        k += dk;
+        if (k >= cpr) {
+            k -= cpr;
+            ++r;
+        }
+    }
+};
+
 // ---------------------------------------------------------------------------------------
 // pass 1a: plain amax over a [rows][cols] bf16 tensor with leading dimension ld
 // ---------------------------------------------------------------------------------------
@@ -75,18 +97,18 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
                                                          uint32_t* __restrict__ flags) {
     __shared__ uint32_t red[8];
     const int64_t cpr = cols >> 3;  // 16-byte chunks per row
-    const int64_t total = rows * cpr;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
-    int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr);
     // four independent loads in flight per iteration
-    for (; c + 3 * stride < total; c += 4 * stride) {
+    while (w.r < rows) {
         uint4 v[4];
+        bool ok[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int64_t cc = c + u * stride;
-            const int64_t r = cc / cpr, k = cc - r * cpr;
-            v[u] = ldg_stream(x + r * ld + (k << 3));
+            ok[u] = w.r < rows;
+            v[u] = ok[u] ? ldg_stream(x + w.r * ld + (w.k << 3)) : make_uint4(0, 0, 0, 0);
+            w.next();
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -96,14 +118,6 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
             m = mag_max2(m, v[u].w);
         }
     }
-    for (; c < total; c += stride) {
-        const int64_t r = c / cpr, k = c - r * cpr;
-        const uint4 v = ldg_stream(x + r * ld + (k << 3));
-        m = mag_max2(m, v.x);
-        m = mag_max2(m, v.y);
-        m = mag_max2(m, v.z);
-        m = mag_max2(m, v.w);
-    }
     uint32_t mag = max(m & 0xFFFFu, m >> 16);
     if (mag >= 0x7F80u) atomicOr(flags, kFlagNonFinite);  // Inf (0x7F80) or NaN
     block_atomic_max(mag << 16, amax_bits, red);
@@ -111,46 +125,40 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
 
 // ---------------------------------------------------------------------------------------
 // pass 1b: plain amax and amax of the 16-point RHT along rows (one read).  A thread takes a
-// 16-row x 8-column patch; rows % 16 == 0, cols % 8 == 0.
+// 16-row x 2-column patch (16 four-byte loads; a warp reads 128 contiguous bytes per row), the
+// column pair transformed as f32x2 pairs.  Few registers per thread keep many patches in flight.
+// rows % 16 == 0, cols % 2 == 0.
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 2) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                       int64_t cols, int64_t ld, uint32_t signs,
+__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                                                       int64_t ld, const SignMasks sm,
                                                        uint32_t* __restrict__ amax_plain_bits,
                                                        uint32_t* __restrict__ amax_rht_bits,
                                                        uint32_t* __restrict__ flags) {
     __shared__ uint32_t red[8];
-    const int64_t cpr = cols >> 3;
+    const int64_t cpr = cols >> 1;
     const int64_t groups = rows >> 4;
-    const int64_t total = groups * cpr;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
     float mr = 0.0f;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += stride) {
-        const int64_t g = u / cpr, k = u - g * cpr;
-        const uint16_t* base = x + (g << 4) * ld + (k << 3);
-        uint4 v[16];
+    for (GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr); w.r < groups; w.next()) {
+        const uint16_t* base = x + (w.r << 4) * ld + (w.k << 1);
+        uint32_t v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = ldg_stream(base + i * ld);
+        for (int i = 0; i < 16; ++i)
+            asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v[i]) : "l"(base + i * ld));
+        uint64_t f[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            m = mag_max2(m, v[i].x);
-            m = mag_max2(m, v[i].y);
-            m = mag_max2(m, v[i].z);
-            m = mag_max2(m, v[i].w);
+            m = mag_max2(m, v[i]);
+            f[i] = bf16x2_to_f2(v[i] ^ sm.m[i]);
         }
-#pragma unroll 1
-        for (int p = 0; p < 4; ++p) {
-            float a[16], b[16];
+        rht16_pairs(f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t w = p == 0 ? v[i].x : p == 1 ? v[i].y : p == 2 ? v[i].z : v[i].w;
-                a[i] = bf16_lo(w);
-                b[i] = bf16_hi(w);
-            }
-            rht16(a, signs);
-            rht16(b, signs);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) mr = fmaxf(mr, fmaxf(fabsf(a[i]), fabsf(b[i])));
+        for (int i = 0; i < 16; i += 2) {
+            float a0, a1, b0, b1;
+            f2_split(f[i], a0, a1);
+            f2_split(f[i + 1], b0, b1);
+            mr = max3_abs(max3_abs(mr, a0, a1), b0, b1);
         }
     }
     uint32_t mag = max(m & 0xFFFFu, m >> 16);
@@ -245,10 +253,33 @@ __device__ __forceinline__ uint32_t e4m3_of_amax(float amax_b, float s_enc) {
     return e4m3_rne_sat(__fmul_rn(__fdiv_rn(amax_b, 6.0f), s_enc));
 }
 
+// Philox4x32-10 of counter (g_lo, g_hi, stream, 0) with the round keys taken from the kernel's
+// parameters (constant-bank operands: no registers held for them)
+__device__ __forceinline__ U4 sr_words_p(const QuantParams& p, uint32_t stream_id, uint64_t g) {
+    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = stream_id, c3 = 0u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ p.key0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ p.key1[r];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+    }
+    return U4{c0, c1, c2, c3};
+}
+
+// four code bytes (each in the low 8 bits of its word) -> one word, byte 0 first
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx, QuantParams p) {
+__global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                     const __grid_constant__ QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x;
     float* s_mult_row = reinterpret_cast<float*>(smem + QuantSmem::mult_row);
     float* s_mult_col = reinterpret_cast<float*>(smem + QuantSmem::mult_col);
     uint8_t* s_tile_code = smem + QuantSmem::tile_code;
@@ -263,7 +294,6 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
     const int64_t ntc = (cols + kTileCols - 1) / kTileCols;
     const int64_t ntiles = ntr * ntc;
     const bool sr_row = ROW && p.sr_row, sr_col = COL && p.sr_col, rht = COL && p.rht_col, b16 = p.block16 != 0;
-    const PhiloxKeys keys = philox_keys(p.sr_seed);
 
     const float senc_r = encode_scale(__uint_as_float(ROW ? *p.amax_row : 0u));
     const float senc_c = encode_scale(__uint_as_float(COL ? *p.amax_col : 0u));
@@ -348,50 +378,55 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
             __syncthreads();
         }
 
-        // ---- R: the ROW form -------------------------------------------------------------------
+        // ---- R: the ROW form, one thread per 1x16 block ----------------------------------------
+        // A warp covers two tile rows (16 blocks each); lanes 4a..4a+3 hold four consecutive
+        // blocks of one row, whose scales leave as one 32-bit word.
         if (ROW) {
 #pragma unroll 1
-            for (int j = tid; j < kTileRows * (kTileCols / 8); j += kQuantThreads) {
-                const int r = j >> 5, ch = j & 31;              // a warp covers one row, 32 chunks
-                const int64_t gr = r_base + r, gc = c_base + ch * 8;
-                const uint4 v = *reinterpret_cast<const uint4*>(sx + r * kTileCols + ch * 8);
+            for (int j = tid; j < kTileRows * (kTileCols / 16); j += kQuantThreads) {
+                const int r = j >> 4, b = j & 15;
+                const int64_t gr = r_base + r, gc = c_base + b * 16;
+                const uint4 v0 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16);
+                const uint4 v1 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16 + 8);
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                 uint32_t code;
                 float mult;
                 if (b16) {
-                    const int tile = ((r >> 4) << 4) + (ch >> 1);
+                    const int tile = ((r >> 4) << 4) + b;
                     code = s_tile_code[tile];
                     mult = s_tile_mult[tile];
                 } else {
-                    uint32_t m = mag_max2(mag_max2(mag_max2(mag_max2(0u, v.x), v.y), v.z), v.w);
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) m = mag_max2(m, w[q]);
                     m = max(m & 0xFFFFu, m >> 16);
-                    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                     code = e4m3_of_amax(__uint_as_float(m << 16), senc_r);
                     mult = s_mult_row[code];
                 }
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                uint32_t packed = 0;
+                const uint64_t mm = f2(mult, mult);
+                uint32_t byte[8];
                 if (sr_row) {
-                    const U4 rw = sr_words(keys, p.stream_row,
-                                           ((uint64_t)(p.row_offset + gr) * (uint64_t)cols + (uint64_t)gc) >> 3);
-                    const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
+                    const uint64_t g0 = ((uint64_t)(p.row_offset + gr) * (uint64_t)cols + (uint64_t)gc) >> 3;
+                    const U4 ra = sr_words_p(p, p.stream_row, g0);
+                    const U4 rb = sr_words_p(p, p.stream_row, g0 + 1);
+                    const uint32_t rr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        packed |= e2m1_sr(__fmul_rn(bf16_lo(w4[q]), mult), rr[q] & 0xFFFFu) << (8 * q);
-                        packed |= e2m1_sr(__fmul_rn(bf16_hi(w4[q]), mult), rr[q] >> 16) << (8 * q + 4);
-                    }
+                    for (int q = 0; q < 8; ++q)
+                        byte[q] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[q]), mm), rr[q] & 0xFFFFu, rr[q] >> 16);
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        packed |= e2m1x2_rne(__fmul_rn(bf16_lo(w4[q]), mult), __fmul_rn(bf16_hi(w4[q]), mult)) << (8 * q);
+                    for (int q = 0; q < 8; ++q) {
+                        float lo, hi;
+                        f2_split(f2_mul(bf16x2_to_f2(w[q]), mm), lo, hi);
+                        byte[q] = e2m1x2_rne(lo, hi);
+                    }
                 }
-                // scales of blocks kb..kb+3 (lanes 8a, 8a+2, 8a+4, 8a+6) -> one 32-bit word
-                uint32_t sw = code;
-                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 8;
-                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 4) << 16;
-                const bool ok = gr < rows && gc < cols;
-                if (ok) {
-                    *reinterpret_cast<uint32_t*>(p.codes_row + gr * (cols >> 1) + (gc >> 1)) = packed;
-                    if ((lane & 7) == 0) {
+                uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
+                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
+                if (gr < rows && gc < cols) {
+                    *reinterpret_cast<uint2*>(p.codes_row + gr * (cols >> 1) + (gc >> 1)) =
+                        make_uint2(pack4(byte[0], byte[1], byte[2], byte[3]), pack4(byte[4], byte[5], byte[6], byte[7]));
+                    if ((b & 3) == 0) {
                         // blocks past `cols` are padding and must read 0
                         const int64_t kb = gc >> 4;
                         const int64_t nv64 = (cols >> 4) - kb;
@@ -403,54 +438,96 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
             }
         }
 
-        // ---- C: the COL form -------------------------------------------------------------------
+        // ---- C: the COL form, one thread per (column pair, 16-row group) -----------------------
+        // The two columns' 16 values arrive as 16 bf16 pairs (one 32-bit shared load per row) and
+        // stay paired through the RHT and the scaling (f32x2 arithmetic).  The SR fields of a form
+        // element are indexed by its position in the form, so each column's 16 elements are two
+        // whole Philox calls.
         if (COL) {
 #pragma unroll 1
-            for (int j = tid; j < 4 * kTileCols; j += kQuantThreads) {
-                const int c = j & (kTileCols - 1), g = j >> 8;   // a warp covers 32 columns of one group
-                float v[16];
+            for (int j = tid; j < 4 * (kTileCols / 2); j += kQuantThreads) {
+                const int cp = j & (kTileCols / 2 - 1), g = j >> 7;   // a warp covers 64 columns of one group
+                const int c = 2 * cp;
+                uint64_t v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = __uint_as_float((uint32_t)sx[(g * 16 + i) * kTileCols + c] << 16);
-                if (rht) rht16(v, p.signs);
-                uint32_t code;
-                float mult;
+                for (int i = 0; i < 16; ++i) {
+                    uint32_t w = *reinterpret_cast<const uint32_t*>(sx + (g * 16 + i) * kTileCols + c);
+                    if (rht) w ^= p.sign_mask2[i];
+                    v[i] = bf16x2_to_f2(w);
+                }
+                if (rht) rht16_pairs(v);
+                uint32_t code0, code1;
+                float mult0, mult1;
                 if (b16) {
                     const int tile = (g << 4) + (c >> 4);
-                    code = s_tile_code[tile];
-                    mult = s_tile_mult[tile];
+                    code0 = code1 = s_tile_code[tile];
+                    mult0 = mult1 = s_tile_mult[tile];
                 } else {
-                    float m = 0.0f;
+                    float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-                    code = e4m3_of_amax(m, senc_c);
-                    mult = s_mult_col[code];
+                    for (int i = 0; i < 16; i += 2) {
+                        float a0, a1, b0, b1;
+                        f2_split(v[i], a0, a1);
+                        f2_split(v[i + 1], b0, b1);
+                        m0 = max3_abs(m0, a0, b0);
+                        m1 = max3_abs(m1, a1, b1);
+                    }
+                    code0 = e4m3_of_amax(m0, senc_c);
+                    code1 = e4m3_of_amax(m1, senc_c);
+                    mult0 = s_mult_col[code0];
+                    mult1 = s_mult_col[code1];
                 }
-                uint32_t c0 = 0, c1 = 0;
+                const uint64_t mm = f2(mult0, mult1);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = f2_mul(v[i], mm);
+                uint32_t out[4];   // column c: out[0..1], column c + 1: out[2..3]
                 if (sr_col) {
                     // form element (column c, row r) has index c * rows_total + row_offset + r; the
                     // block's first row is a multiple of 16, so its 16 fields are Philox calls i0/8, i0/8 + 1
                     const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)p.rows_total +
                                          (uint64_t)(p.row_offset + r_base + g * 16)) >> 3;
-                    const U4 w0 = sr_words(keys, p.stream_col, g0);
-                    const U4 w1 = sr_words(keys, p.stream_col, g0 + 1);
-                    const uint32_t rw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    const uint64_t g1 = g0 + ((uint64_t)p.rows_total >> 3);   // column c + 1
+                    uint32_t nib[16];   // per row i: column c's code in bits [0,4), column c + 1's in [4,8)
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t r16 = (i & 1) ? (rw[i >> 1] >> 16) : (rw[i >> 1] & 0xFFFFu);
-                        const uint32_t n = e2m1_sr(__fmul_rn(v[i], mult), r16);
-                        if (i < 8) c0 |= n << (4 * i);
-                        else c1 |= n << (4 * (i - 8));
+                    for (int h = 0; h < 2; ++h) {   // rows 8h .. 8h + 7: one Philox call per column
+                        const U4 a = sr_words_p(p, p.stream_col, g0 + h), b = sr_words_p(p, p.stream_col, g1 + h);
+                        const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t r0 = (i & 1) ? (ra[i >> 1] >> 16) : (ra[i >> 1] & 0xFFFFu);
+                            const uint32_t r1 = (i & 1) ? (rb[i >> 1] >> 16) : (rb[i >> 1] & 0xFFFFu);
+                            nib[8 * h + i] = e2m1_sr_pair(v[8 * h + i], r0, r1);
+                        }
                     }
+                    // rows 2q, 2q + 1 -> byte q of each column's codes
+                    uint32_t bc0[8], bc1[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        bc0[q] = (nib[2 * q] & 15u) | ((nib[2 * q + 1] & 15u) << 4);
+                        bc1[q] = (nib[2 * q] >> 4) | (nib[2 * q + 1] & 0xF0u);
+                    }
+                    out[0] = pack4(bc0[0], bc0[1], bc0[2], bc0[3]);
+                    out[1] = pack4(bc0[4], bc0[5], bc0[6], bc0[7]);
+                    out[2] = pack4(bc1[0], bc1[1], bc1[2], bc1[3]);
+                    out[3] = pack4(bc1[4], bc1[5], bc1[6], bc1[7]);
                 } else {
+                    uint32_t bc0[8], bc1[8];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        c0 |= e2m1x2_rne(__fmul_rn(v[2 * q], mult), __fmul_rn(v[2 * q + 1], mult)) << (8 * q);
-                        c1 |= e2m1x2_rne(__fmul_rn(v[8 + 2 * q], mult), __fmul_rn(v[9 + 2 * q], mult)) << (8 * q);
+                    for (int q = 0; q < 8; ++q) {
+                        float a0, a1, b0, b1;
+                        f2_split(v[2 * q], a0, a1);
+                        f2_split(v[2 * q + 1], b0, b1);
+                        bc0[q] = e2m1x2_rne(a0, b0);
+                        bc1[q] = e2m1x2_rne(a1, b1);
                     }
+                    out[0] = pack4(bc0[0], bc0[1], bc0[2], bc0[3]);
+                    out[1] = pack4(bc0[4], bc0[5], bc0[6], bc0[7]);
+                    out[2] = pack4(bc1[0], bc1[1], bc1[2], bc1[3]);
+                    out[3] = pack4(bc1[4], bc1[5], bc1[6], bc1[7]);
                 }
                 const bool grp_ok = r_base + g * 16 < rows;
-                *reinterpret_cast<uint2*>(s_codes + (g * kTileCols + c) * 8) = make_uint2(c0, c1);
-                s_scales[g * kTileCols + c] = grp_ok ? (uint8_t)code : (uint8_t)0;
+                *reinterpret_cast<uint4*>(s_codes + (g * kTileCols + c) * 8) = make_uint4(out[0], out[1], out[2], out[3]);
+                *reinterpret_cast<uint16_t*>(s_scales + g * kTileCols + c) = grp_ok ? (uint16_t)(code0 | (code1 << 8)) : (uint16_t)0;
             }
             __syncthreads();
             // ---- S: staged COL codes and scales to global memory ---------------------------------
@@ -489,6 +566,226 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_tile_kernel(const __gr
         __syncthreads();   // the buffer and the staging areas are free for the next tile
     }
     // copies issued but never consumed (only after a timeout) must land before the CTA exits
+    if (tid == 0) {
+        for (int k = consumed; k < issued; ++k) q_wait(smem_addr(&bars[k & 1]), (uint32_t)(k >> 1) & 1u, 2000000000ull);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// MXFP4, the pages' comparison format (gist.science 2.A): blocks of 32 elements along K, one
+// UE8M0 scale 2^E per block with E = floor(log2 amax_b) - 2 (2 = the largest E2M1 exponent;
+// stored as E + 127, clamped to [0, 254]; an all-zero block gets 0), no tensor scale and so no
+// amax pass.  Elements u = v * 2^-E (one exact power-of-two product, rounded only if it lands
+// below the normal range) go through the same E2M1 encoders as NVFP4, RNE or SR; SR fields are
+// indexed by the element's position in the form.  The same TMA-fed persistent tile walk as the
+// NVFP4 quantizer, one form per call:
+//   ROW form: one thread per 1x32 block (four 16-byte shared loads), 16 code bytes per store;
+//   COL form: one thread per (column pair, 32-row group): the 32 bf16 pairs give both columns'
+//             block maxima by packed integer max, then the codes are staged and leave as rows.
+// ---------------------------------------------------------------------------------------
+// UE8M0 code of a block whose largest magnitude has bf16 bits m (sign cleared)
+__device__ __forceinline__ uint32_t ue8m0_of_mag(uint32_t m) {
+    if (m == 0) return 0u;
+    const int e = (int)(m >> 7);
+    const int fl = e ? e - 127 : (31 - __clz((int)(m & 0x7Fu))) - 133;   // floor(log2 amax_b)
+    return (uint32_t)min(max(fl + 125, 0), 254);
+}
+// 2^-E = 2^(127 - code), exact (2^-127 is the one subnormal case)
+__device__ __forceinline__ float ue8m0_inv(uint32_t code) {
+    return __uint_as_float(code == 254u ? 0x00400000u : (254u - code) << 23);
+}
+
+__device__ __forceinline__ U4 mx_words(const MxParams& p, uint64_t g) {
+    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = p.stream_id, c3 = 0u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ p.key0[r], n2 = (uint32_t)(p0 >> 32) ^ c3 ^ p.key1[r];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+    }
+    return U4{c0, c1, c2, c3};
+}
+
+template <bool COLF>
+__global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                      const __grid_constant__ MxParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QuantSmem::bars);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + QuantSmem::bars + 16);
+    uint8_t* s_codes = smem + QuantSmem::codes;
+    uint8_t* s_scales = smem + QuantSmem::scales;
+    const int64_t rows = p.rows, cols = p.cols;
+    const int64_t ntr = (rows + kTileRows - 1) / kTileRows;
+    const int64_t ntc = (cols + kTileCols - 1) / kTileCols;
+    const int64_t ntiles = ntr * ntc;
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[0])) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[1])) : "memory");
+        *s_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    int64_t it = blockIdx.x;
+    if (tid == 0 && it < ntiles)
+        q_load_tile(smem_addr(smem + QuantSmem::x0), &tmx, (int32_t)((it % ntc) * kTileCols), (int32_t)((it / ntc) * kTileRows),
+                    smem_addr(&bars[0]));
+    int issued = (it < ntiles) ? 1 : 0, consumed = 0;
+    for (int local = 0; it < ntiles; it += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const int64_t tr = it / ntc, tc = it - tr * ntc;
+        if (tid == 0 && it + gridDim.x < ntiles) {
+            const int64_t n = it + gridDim.x;
+            q_load_tile(smem_addr(smem + (buf ? QuantSmem::x0 : QuantSmem::x1)), &tmx, (int32_t)((n % ntc) * kTileCols),
+                        (int32_t)((n / ntc) * kTileRows), smem_addr(&bars[buf ^ 1]));
+            ++issued;
+        }
+        if (!q_wait(smem_addr(&bars[buf]), (uint32_t)(local >> 1) & 1u, 2000000000ull)) *s_abort = 1u;
+        __syncthreads();
+        if (*s_abort) {
+            if (tid == 0) atomicOr(p.flags, kFlagTimeout);
+            break;
+        }
+        ++consumed;
+        const uint16_t* sx = reinterpret_cast<const uint16_t*>(smem + (buf ? QuantSmem::x1 : QuantSmem::x0));
+        const int64_t r_base = tr * kTileRows, c_base = tc * kTileCols;
+        if (!COLF) {
+            // ---- ROW form: one thread per 1x32 block; lanes 4a..4a+3 hold four blocks of one row
+#pragma unroll 1
+            for (int j = tid; j < kTileRows * (kTileCols / 32); j += kQuantThreads) {
+                const int r = j >> 3, b = j & 7;
+                const int64_t gr = r_base + r, gc = c_base + b * 32;
+                uint32_t w[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 32 + 8 * q);
+                    w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                }
+                uint32_t m = 0;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) m = mag_max2(m, w[q]);
+                const uint32_t code = ue8m0_of_mag(max(m & 0xFFFFu, m >> 16));
+                const float inv = ue8m0_inv(code);
+                const uint64_t mm = f2(inv, inv);
+                uint32_t byte[16];
+                if (p.sr) {
+                    const uint64_t g0 = ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const U4 rw = mx_words(p, g0 + c);
+                        const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            byte[4 * c + q] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), rr[q] & 0xFFFFu, rr[q] >> 16);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        float lo, hi;
+                        f2_split(f2_mul(bf16x2_to_f2(w[q]), mm), lo, hi);
+                        byte[q] = e2m1x2_rne(lo, hi);
+                    }
+                }
+                uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
+                sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
+                if (gr < rows && gc < cols) {
+                    *reinterpret_cast<uint4*>(p.codes + gr * (cols >> 1) + (gc >> 1)) =
+                        make_uint4(pack4(byte[0], byte[1], byte[2], byte[3]), pack4(byte[4], byte[5], byte[6], byte[7]),
+                                   pack4(byte[8], byte[9], byte[10], byte[11]), pack4(byte[12], byte[13], byte[14], byte[15]));
+                    if ((b & 3) == 0) {
+                        const int64_t kb = gc >> 5;
+                        const int64_t nv64 = (cols >> 5) - kb;
+                        const int nvalid = nv64 < 4 ? (int)nv64 : 4;
+                        const uint32_t keep = nvalid >= 4 ? 0xFFFFFFFFu : ((1u << (8 * nvalid)) - 1u);
+                        *reinterpret_cast<uint32_t*>(p.scales + scale_offset(gr, kb, p.nkt)) = sw & keep;
+                    }
+                }
+            }
+        } else {
+            // ---- COL form: one thread per (column pair, 32-row group) -------------------------
+            {
+                const int cp = tid & (kTileCols / 2 - 1), g = tid >> 7;
+                const int c = 2 * cp;
+                uint32_t w[32];
+                uint32_t m = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    w[i] = *reinterpret_cast<const uint32_t*>(sx + (g * 32 + i) * kTileCols + c);
+                    m = mag_max2(m, w[i]);
+                }
+                const uint32_t code0 = ue8m0_of_mag(m & 0xFFFFu), code1 = ue8m0_of_mag(m >> 16);
+                const uint64_t mm = f2(ue8m0_inv(code0), ue8m0_inv(code1));
+                uint32_t out[8];   // column c: out[0..3], column c + 1: out[4..7]
+                if (p.sr) {
+                    const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)rows + (uint64_t)(r_base + g * 32)) >> 3;
+                    const uint64_t g1 = g0 + ((uint64_t)rows >> 3);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {   // rows 8h .. 8h + 7: one Philox call per column
+                        const U4 a = mx_words(p, g0 + h), bw = mx_words(p, g1 + h);
+                        const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {bw.x, bw.y, bw.z, bw.w};
+                        uint32_t nib[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t r0 = (i & 1) ? (ra[i >> 1] >> 16) : (ra[i >> 1] & 0xFFFFu);
+                            const uint32_t r1 = (i & 1) ? (rb[i >> 1] >> 16) : (rb[i >> 1] & 0xFFFFu);
+                            nib[i] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), r0, r1);
+                        }
+                        uint32_t b0[4], b1[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            b0[q] = (nib[2 * q] & 15u) | ((nib[2 * q + 1] & 15u) << 4);
+                            b1[q] = (nib[2 * q] >> 4) | (nib[2 * q + 1] & 0xF0u);
+                        }
+                        out[h] = pack4(b0[0], b0[1], b0[2], b0[3]);
+                        out[4 + h] = pack4(b1[0], b1[1], b1[2], b1[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t b0[4], b1[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float a0, a1, c0v, c1v;
+                            f2_split(f2_mul(bf16x2_to_f2(w[8 * h + 2 * q]), mm), a0, a1);
+                            f2_split(f2_mul(bf16x2_to_f2(w[8 * h + 2 * q + 1]), mm), c0v, c1v);
+                            b0[q] = e2m1x2_rne(a0, c0v);
+                            b1[q] = e2m1x2_rne(a1, c1v);
+                        }
+                        out[h] = pack4(b0[0], b0[1], b0[2], b0[3]);
+                        out[4 + h] = pack4(b1[0], b1[1], b1[2], b1[3]);
+                    }
+                }
+                const bool grp_ok = r_base + g * 32 < rows;
+                *reinterpret_cast<uint4*>(s_codes + (g * kTileCols + c) * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+                *reinterpret_cast<uint4*>(s_codes + (g * kTileCols + c + 1) * 16) = make_uint4(out[4], out[5], out[6], out[7]);
+                *reinterpret_cast<uint16_t*>(s_scales + g * kTileCols + c) = grp_ok ? (uint16_t)(code0 | (code1 << 8)) : (uint16_t)0;
+            }
+            __syncthreads();
+            // staged codes and scales to global memory: per column 16 code bytes and one scale per group
+            const int64_t rem = (rows - r_base) >> 5;
+            const int ngroups = rem < 2 ? (int)rem : 2;
+            const int64_t kbytes = rows >> 1;
+#pragma unroll 1
+            for (int j = tid; j < 2 * kTileCols; j += kQuantThreads) {
+                const int c = j >> 1, g = j & 1;
+                if (c_base + c < cols && g < ngroups)
+                    *reinterpret_cast<uint4*>(p.codes + (c_base + c) * kbytes + (r_base >> 1) + g * 16) =
+                        *reinterpret_cast<const uint4*>(s_codes + (g * kTileCols + c) * 16);
+            }
+            for (int c = tid; c < kTileCols; c += kQuantThreads) {
+                if (c_base + c < cols) {
+                    uint8_t* dst = p.scales + scale_offset(c_base + c, r_base >> 5, p.nkt);
+                    dst[0] = s_scales[c];
+                    if (ngroups > 1) dst[1] = s_scales[kTileCols + c];
+                }
+            }
+        }
+        __syncthreads();
+    }
     if (tid == 0) {
         for (int k = consumed; k < issued; ++k) q_wait(smem_addr(&bars[k & 1]), (uint32_t)(k >> 1) & 1u, 2000000000ull);
     }
@@ -551,10 +848,10 @@ cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int
 
 cudaError_t launch_amax_rht(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t signs,
                             uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags, cudaStream_t s) {
-    const int64_t units = (rows >> 4) * (cols >> 3);
+    const int64_t units = (rows >> 4) * (cols >> 1);
     if (units == 0) return cudaSuccess;
-    amax_rht_kernel<<<grid_for(units, 256, 2), 256, 0, s>>>(x, rows, cols, ld, signs, amax_plain, amax_rht,
-                                                           flags);
+    amax_rht_kernel<<<grid_for(units, 256, 8), 256, 0, s>>>(x, rows, cols, ld, sign_masks(signs), amax_plain,
+                                                           amax_rht, flags);
     return cudaGetLastError();
 }
 
@@ -586,8 +883,17 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    QuantParams q = p;
+    for (int j = 0; j < 16; ++j) q.sign_mask2[j] = ((p.signs >> j) & 1u) ? 0x80008000u : 0u;
+    uint32_t k0 = (uint32_t)p.sr_seed, k1 = (uint32_t)(p.sr_seed >> 32);
+    for (int r = 0; r < 10; ++r) {   // the Philox4x32-10 key schedule (Salmon et al., SC'11)
+        q.key0[r] = k0;
+        q.key1[r] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
     const int smem = QuantSmem::bytes;
-    void (*kern)(const CUtensorMap, QuantParams) =
+    void (*kern)(const CUtensorMap, const QuantParams) =
         row && col ? quantize_tile_kernel<true, true> : row ? quantize_tile_kernel<true, false> : quantize_tile_kernel<false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
     if (e != cudaSuccess) return e;
@@ -598,7 +904,42 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
     if (per_sm < 1) per_sm = 1;
     const int64_t cap = (int64_t)sms * per_sm;
     const int grid = (int)(ntiles < cap ? ntiles : cap);
-    kern<<<grid, kQuantThreads, smem, s>>>(map, p);
+    kern<<<grid, kQuantThreads, smem, s>>>(map, q);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_seed, cudaStream_t s) {
+    const int64_t ntiles = ((p.rows + kTileRows - 1) / kTileRows) * ((p.cols + kTileCols - 1) / kTileCols);
+    if (ntiles == 0) return cudaSuccess;
+    auto fn = q_encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)p.cols, (cuuint64_t)p.rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(p.ld * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)kTileCols, (cuuint32_t)kTileRows};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(p.x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    MxParams q = p;
+    uint32_t k0 = (uint32_t)sr_seed, k1 = (uint32_t)(sr_seed >> 32);
+    for (int r = 0; r < 10; ++r) {   // the Philox4x32-10 key schedule
+        q.key0[r] = k0;
+        q.key1[r] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    void (*kern)(const CUtensorMap, const MxParams) = column_form ? quantize_mx_kernel<true> : quantize_mx_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantThreads, QuantSmem::bytes);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t cap = (int64_t)sms * per_sm;
+    kern<<<(int)(ntiles < cap ? ntiles : cap), kQuantThreads, QuantSmem::bytes, s>>>(map, q);
     return cudaGetLastError();
 }
 

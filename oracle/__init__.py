@@ -87,6 +87,10 @@ def lib():
         L.ora_ue8m0_of_amax.restype = c.c_uint8
         L.ora_quantize_mx.argtypes = [u16p, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_uint64, c.c_uint32, u8p, u8p]
         L.ora_quantize_mx.restype = c.c_int
+        L.ora_dequantize_mx.argtypes = [u8p, u8p, c.c_int64, c.c_int64, f64p]
+        L.ora_dequantize_mx.restype = None
+        L.ora_mx_scales_swizzle.argtypes = [u8p, c.c_int64, c.c_int64, u8p]
+        L.ora_mx_scales_swizzle.restype = None
         _LIB = L
     return _LIB
 
@@ -318,3 +322,41 @@ def quantize_mx(x_bits: np.ndarray, mode: int = RNE, sr_seed: int = 0, stream_id
     if st != 0:
         raise ValueError(f"ora_quantize_mx: status {st}")
     return codes, scales
+
+
+def dequantize_mx(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """MXFP4 form -> fp64 values [R][K]: E2M1(code) * 2^(scale - 127), exact."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    R, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((R, K), np.float64)
+    lib().ora_dequantize_mx(_p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8), R, K, _p(out, ctypes.c_double))
+    return out
+
+
+def mx_scales_swizzled(scales: np.ndarray, K: int) -> np.ndarray:
+    """Row-major MXFP4 scales [R][K/32] in the 128x4 tile layout of the block-scaled MMA."""
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    R = scales.shape[0]
+    sw = np.empty(((R + 127) // 128) * 128 * ((K // 32 + 3) // 4) * 4, np.uint8)
+    lib().ora_mx_scales_swizzle(_p(scales, ctypes.c_uint8), R, K, _p(sw, ctypes.c_uint8))
+    return sw
+
+
+def gemm_mx(a_codes, a_scales, b_codes, b_scales):
+    """D = A * B^T in fp64 over dequantized MXFP4 operands (numpy's matmul as the dot-product
+    step), plus sum_k |a_ik b_jk|."""
+    A, B = dequantize_mx(a_codes, a_scales), dequantize_mx(b_codes, b_scales)
+    return A @ B.T, np.abs(A) @ np.abs(B).T
+
+
+# ---------------------------------------------------------------------------------------
+# BF16 GEMM of the high-precision layers: the plain definition, in fp64
+# ---------------------------------------------------------------------------------------
+def gemm_bf16(a_bits: np.ndarray, b_bits: np.ndarray):
+    """D = A * B^T in fp64 over bf16 operands given as uint16 bit patterns ([M][K], [N][K]);
+    every bf16 value and every product is exact in fp64 (numpy's matmul as the dot-product step).
+    Returns D and sum_k |a_ik b_jk|."""
+    A = bf16_bits_to_f32(a_bits).astype(np.float64)
+    B = bf16_bits_to_f32(b_bits).astype(np.float64)
+    return A @ B.T, np.abs(A) @ np.abs(B).T

@@ -694,3 +694,29 @@ int ora_quantize_mx(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
     }
     return ORA_OK;
 }
+
+/* MXFP4 dequantize: value = E2M1(code) * 2^(scale - 127), exact in fp64 (codes [R][K/2] with the
+   even element in the low nibble, UE8M0 scales [R][K/32] row-major; scale 255 is NaN and never
+   produced by ora_quantize_mx). */
+void ora_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t K, double* out)
+{
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            const uint8_t byte = codes[r * (K / 2) + k / 2];
+            const uint8_t nib = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
+            const double scale = ldexp(1.0, (int)scales[r * (K / 32) + k / 32] - 127);
+            out[r * K + k] = ora_e2m1_value(nib) * scale;
+        }
+}
+
+/* The MXFP4 scales [R][K/32] in the 128x4 tiles the block-scaled MMA reads: entry (r, kb) at
+   ((r/128)*ceil(K/128) + kb/4)*512 + (r%32)*16 + ((r/32)%4)*4 + kb%4, padding 0 (sw holds
+   ceil(R/128)*128 * ceil(K/128)*4 bytes). */
+void ora_mx_scales_swizzle(const uint8_t* scales, int64_t R, int64_t K, uint8_t* sw)
+{
+    const int64_t nkt = (K / 32 + 3) / 4;
+    memset(sw, 0, (size_t)(((R + 127) / 128) * 128 * nkt * 4));
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t kb = 0; kb < K / 32; ++kb)
+            sw[((r / 128) * nkt + kb / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + (kb % 4)] = scales[r * (K / 32) + kb];
+}

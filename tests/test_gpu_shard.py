@@ -110,3 +110,29 @@ def test_shard_wgrad_partials_reduce_to_the_whole_batch_dw(T, d, n, shards):
     for a, b in zip(dyc, xc):
         total += m.nvfp4_gemm(a, b, out_dtype=torch.float32)
     check_gemm(total.cpu().numpy(), ref, sabs, False, f"sum of {shards} shard dW partials")
+
+
+def test_dp_linear_on_one_rank_equals_the_linear_layer():
+    # DPLinear through a one-rank NCCL group: the all-reduce is the identity and the reduce-scatter
+    # keeps every row, so Y, dX and dW equal nvfp4_linear_fwd/bwd bit for bit
+    import torch.distributed as dist
+    m = nv()
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        T, d, n = 256, 320, 512
+        x, w, dy = (to_device_bf16(t) for t in (synth.activations(T, d, seed=0, outlier_frac=0.01),
+                                                 synth.weights(n, d, seed=1), synth.grad_output(T, n, seed=2)))
+        ctx = m.LinearContext(T, d, n, rht_seed=3)
+        y1 = m.nvfp4_linear_fwd(ctx, x, w)
+        dx1, dw1 = m.nvfp4_linear_bwd(ctx, dy, 4)
+        dp = m.DPLinear(T, d, n, rht_seed=3)
+        y2 = dp.fwd(x, w)
+        dx2 = dp.bwd(dy, 4)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2) and torch.equal(dx1, dx2) and torch.equal(dw1, dp.dw)
+    finally:
+        dist.destroy_process_group()

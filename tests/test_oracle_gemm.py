@@ -77,3 +77,29 @@ def test_rht_cancels_in_wgrad(ora):
     ref = f(dy).T.astype(np.float64) @ f(x).astype(np.float64)
     got = rot(dy).astype(np.float64) @ rot(x).astype(np.float64).T
     assert np.allclose(got, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
+def test_bf16_gemm_is_the_exact_product(ora):
+    # the BF16 path's oracle GEMM: integer-valued bf16 operands make every product and sum an exact
+    # integer, checked against Python's arbitrary-precision integers; a fractional case against
+    # Fraction arithmetic on the decoded bf16 values
+    from fractions import Fraction
+    import torch
+    g = torch.Generator().manual_seed(3)
+    a = torch.randint(-64, 65, (7, 40), generator=g).to(torch.bfloat16)
+    b = torch.randint(-64, 65, (5, 40), generator=g).to(torch.bfloat16)
+    d, s = ora.gemm_bf16(synth.bf16_bits(a), synth.bf16_bits(b))
+    ai, bi = a.to(torch.int64).tolist(), b.to(torch.int64).tolist()
+    for i in range(7):
+        for j in range(5):
+            assert d[i, j] == sum(x * y for x, y in zip(ai[i], bi[j]))
+            assert s[i, j] == sum(abs(x * y) for x, y in zip(ai[i], bi[j]))
+    x = (torch.randn(3, 24, generator=g) * 3).to(torch.bfloat16)
+    w = (torch.randn(4, 24, generator=g) * 0.02).to(torch.bfloat16)
+    d, _ = ora.gemm_bf16(synth.bf16_bits(x), synth.bf16_bits(w))
+    xf = [[Fraction(float(v)) for v in row] for row in x.float().tolist()]
+    wf = [[Fraction(float(v)) for v in row] for row in w.float().tolist()]
+    for i in range(3):
+        for j in range(4):
+            exact = sum(p * q for p, q in zip(xf[i], wf[j]))
+            assert abs(Fraction(d[i, j]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)

@@ -130,3 +130,37 @@ def test_hand_worked_block(ora):
     codes, scales = ora.quantize_mx(_bits(v)[None, :])
     assert scales.tolist() == [[126]]
     assert codes[0, 0] == 0xC7 and codes[0, 1] == 0x02 and not codes[0, 2:].any()
+
+
+def test_mx_dequantize_and_gemm_match_independent_decoder(ora):
+    # the oracle's MXFP4 dequantizer and fp64 GEMM against ml_dtypes' E2M1 and E8M0 decoders
+    import ml_dtypes
+    x = synth.bf16_bits(synth.activations(48, 256, seed=3, outlier_frac=0.05))
+    w = synth.bf16_bits(synth.weights(40, 256, seed=4))
+    (ca, sa), (cb, sb) = ora.quantize_mx(x), ora.quantize_mx(w, mode=SR, sr_seed=5, stream_id=1)
+
+    def ml(codes, scales):
+        nib = np.empty((codes.shape[0], codes.shape[1] * 2), np.uint8)
+        nib[:, 0::2], nib[:, 1::2] = codes & 15, codes >> 4
+        vals = nib.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+        return vals * scales.view(ml_dtypes.float8_e8m0fnu).astype(np.float64).repeat(32, axis=1)
+
+    A, B = ml(ca, sa), ml(cb, sb)
+    assert np.array_equal(ora.dequantize_mx(ca, sa), A)
+    d, s = ora.gemm_mx(ca, sa, cb, sb)
+    ref = A @ B.T
+    assert np.allclose(d, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    assert np.allclose(s, np.abs(A) @ np.abs(B).T, rtol=1e-12)
+
+
+def test_mx_swizzle_places_every_scale_once(ora):
+    # the tile layout is a bijection from (row, block) onto the non-padding bytes: tag every
+    # scale with a distinct value and read each back at its closed-form offset
+    R, K = 200, 96 * 4
+    sc = (np.arange(R * (K // 32)) % 251 + 1).astype(np.uint8).reshape(R, K // 32)
+    sw = ora.mx_scales_swizzled(sc, K)
+    nkt = (K // 32 + 3) // 4
+    rr, kk = np.meshgrid(np.arange(R), np.arange(K // 32), indexing="ij")
+    off = ((rr // 128) * nkt + kk // 4) * 512 + (rr % 32) * 16 + ((rr // 32) % 4) * 4 + kk % 4
+    assert np.array_equal(sw[off], sc)
+    assert np.count_nonzero(sw) == sc.size
