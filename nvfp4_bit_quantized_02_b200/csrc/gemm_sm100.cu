@@ -1043,16 +1043,24 @@ static cudaError_t ensure_smem_attr(const void* kernel, int bytes, std::atomic<u
     return e;
 }
 
+// SM count of the current device, looked up once per device
+static int sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
 template <bool MX>
 static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
                                const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                                void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
                                cudaStream_t stream) {
-    static std::atomic<uint64_t> attr_1sm{0};
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_kernel<MX>), kGemmSmem, attr_1sm)) return e;
-    CUtensorMap ta, tb;
-    if (!make_code_map(&ta, a_codes, M, K, kBM) || !make_code_map(&tb, b_codes, N, K, kBN))
-        return cudaErrorInvalidValue;
     GemmParams p;
     p.sfa = a_scales;
     p.sfb = b_scales;
@@ -1074,9 +1082,7 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     p.group_n = (M <= N) ? 1 : 0;   // operands are M x K and N x K: sweep the smaller one
     p.flags = flags;
     p.budget_ns = budget_ns;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     // SM-pair tiles for M >= 256 (fewer operand bytes per SM per K block, a deeper ring);
     // NVFP4_GEMM_VARIANT=1sm selects the 1-SM kernel for every shape (read on every call)
     const char* variant = getenv("NVFP4_GEMM_VARIANT");
@@ -1098,6 +1104,11 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2, p);
         return cudaGetLastError();
     }
+    static std::atomic<uint64_t> attr_1sm{0};
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_kernel<MX>), kGemmSmem, attr_1sm)) return e;
+    CUtensorMap ta, tb;
+    if (!make_code_map(&ta, a_codes, M, K, kBM) || !make_code_map(&tb, b_codes, N, K, kBN))
+        return cudaErrorInvalidValue;
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     CUtensorMap td;
@@ -1162,9 +1173,7 @@ cudaError_t launch_gemm_bf16(const uint16_t* a, int64_t lda, const uint16_t* b, 
     p.group_n = (M <= N) ? 1 : 0;
     p.flags = flags;
     p.budget_ns = budget_ns;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     CUtensorMap ta, tb, td;
     if (!make_bf16_map(&ta, a, M, K, lda) || !make_bf16_map(&tb, b, N, K, ldb) || !make_out_map(&td, d, M, N, ldd, out_fp32))
         return cudaErrorInvalidValue;

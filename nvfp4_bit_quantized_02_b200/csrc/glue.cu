@@ -106,7 +106,7 @@ __device__ __forceinline__ uint4 gelu_chunk(const uint4 x, const uint4 d) {
 }
 
 template <bool BWD>
-__global__ void __launch_bounds__(kGaThreads) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
+__global__ void __launch_bounds__(kGaThreads, 4) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
                                                             uint16_t* __restrict__ out, int64_t rows, int64_t cols,
                                                             const SignMasks sm, uint32_t* __restrict__ amax_plain,
                                                             uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
@@ -254,7 +254,7 @@ cudaError_t launch_gelu_amax(bool bwd, const uint16_t* h, const uint16_t* dg, ui
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 3;   // resident CTAs (16 KB of shared memory, <= 80 registers each)
+    const int64_t cap = (int64_t)sms * 4;   // resident CTAs (16 KB of shared memory, <= 64 registers each)
     const int grid = (int)(tiles < cap ? tiles : cap);
     if (bwd)
         gelu_amax_kernel<true><<<grid, kGaThreads, 0, s>>>(h, dg, out, rows, cols, sign_masks(signs), amax_plain, amax_rht,

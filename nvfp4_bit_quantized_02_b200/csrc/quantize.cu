@@ -99,7 +99,29 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
     const int64_t cpr = cols >> 3;  // 16-byte chunks per row
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
+    if (ld == cols) {
+        // contiguous rows: one flat array of 16-byte chunks, four loads in flight per iteration
+        const int64_t total = rows * cpr;
+        int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; c + 3 * stride < total; c += 4 * stride) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = ldg_stream(x + ((c + u * stride) << 3));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                m = mag_max2(m, v[u].x);
+                m = mag_max2(m, v[u].y);
+                m = mag_max2(m, v[u].z);
+                m = mag_max2(m, v[u].w);
+            }
+        }
+        for (; c < total; c += stride) {
+            const uint4 v = ldg_stream(x + (c << 3));
+            m = mag_max2(mag_max2(mag_max2(mag_max2(m, v.x), v.y), v.z), v.w);
+        }
+    }
     GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr);
+    if (ld == cols) w.r = rows;   // done above
     // four independent loads in flight per iteration
     while (w.r < rows) {
         uint4 v[4];
