@@ -44,8 +44,8 @@ FP4_FLOP_PER_CLK = 2 * 16384 * 148
 # of one ncu capture of the SM-pair GEMM at this layer's shapes, valid for the GEMM source it was
 # taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
 GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
-GEMM_TRAFFIC = {"sha256": "1b1ff1cb88ee135cae6fadffa2b5882b18ff9143af5e688ab53806a543826b35",
-                "bytes_per_launch": 486.5e6}
+GEMM_TRAFFIC = {"sha256": "e3b2bc5b716eab8373581443e49d61f2ef5f5d7a5e701936d68588cc80b3f2e1",
+                "bytes_per_launch": 484.9e6}
 
 
 def gemm_traffic():
@@ -344,6 +344,7 @@ def run_ours(args, rank, world, local_rank):
                        "event-ordered streams"}
 
     ffn = ffn_fields(args, world, dev, dist, flush) if args.ffn else None
+    variants = variant_fields(args, dev, flush, x, w, dy) if args.variants else None
     if rank != 0:
         return None
     clocks = clk.summary()
@@ -383,8 +384,10 @@ def run_ours(args, rank, world, local_rank):
         "calls_ms_per_step": calls_ms_per_step,
         "clocks": clocks,
         "e2e": e2e,
-        "c1_small_fprop": c1_latency(nv, dev),
+        "c1_small_fprop": c1_latency(nv, dev) if args.c1 else None,
         "ffn_step": ffn,
+        "mxfp4_step": variants["mxfp4_step"] if variants else None,
+        "bf16_step": variants["bf16_step"] if variants else None,
         "gpu_launches": launches_per_step * args.steps,
         "impl": "ours",
     }
@@ -526,6 +529,70 @@ def run_ffn(args, rank, world, local_rank):
     }
 
 
+def time_calls(calls, steps, warmup, flush):
+    """Mean device time of each named call of a step (events between calls on the current stream)
+    and of the whole step, over `steps` steps after `warmup`, L2 flushed between steps."""
+    for i in range(warmup):
+        for _, fn in calls:
+            fn(1000 + i)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    for k in range(steps):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record()
+        for i, (_, fn) in enumerate(calls):
+            fn(k)
+            ev[k][i + 1].record()
+    torch.cuda.synchronize()
+    per = {name: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps))
+           for i, (name, _) in enumerate(calls)}
+    return per, statistics.mean(ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps))
+
+
+def variant_fields(args, dev, flush, x, w, dy) -> dict:
+    """The same layer step in the pages' comparison format (MXFP4: six single-pass quantizes and
+    three kind::mxf4 GEMMs) and on the BF16 path of the high-precision layers (three kind::f16
+    GEMMs and the transposes of their K-major operands)."""
+    import nvfp4_bit_quantized_02_b200 as nv
+    ws = nv.Workspace(dev)
+    f = {k: nv.MXTensor.empty(R, K, dev) for k, R, K in (("xr", T_TOK, D_IN), ("xc", D_IN, T_TOK), ("wr", D_OUT, D_IN),
+                                                         ("wc", D_IN, D_OUT), ("dyr", T_TOK, D_OUT),
+                                                         ("dyc", D_OUT, T_TOK))}
+    y = torch.empty((T_TOK, D_OUT), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((T_TOK, D_IN), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
+    mq = nv.nvfp4_mx_quantize
+    mx_calls = [
+        ("quantize X (row, column)", lambda k: (mq(x, 0, out=f["xr"], ws=ws), mq(x, 1, out=f["xc"], ws=ws))),
+        ("quantize W (row, column)", lambda k: (mq(w, 0, out=f["wr"], ws=ws), mq(w, 1, out=f["wc"], ws=ws))),
+        ("fprop", lambda k: nv.nvfp4_mx_gemm(f["xr"], f["wr"], out=y, ws=ws)),
+        ("quantize dY (row, column; SR)", lambda k: (mq(dy, 0, nv.SR, k, 1, out=f["dyr"], ws=ws),
+                                                     mq(dy, 1, nv.SR, k, 2, out=f["dyc"], ws=ws))),
+        ("dgrad", lambda k: nv.nvfp4_mx_gemm(f["dyr"], f["wc"], out=dx, ws=ws)),
+        ("wgrad", lambda k: nv.nvfp4_mx_gemm(f["dyc"], f["xc"], out=dw, ws=ws)),
+    ]
+    per, ms = time_calls(mx_calls, args.steps, args.warmup, flush)
+    out = {"mxfp4_step": {
+        "value": FLOP_STEP / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms, "per_call_ms": per,
+        "gemm_tflops": {g: FLOP_GEMM / per[g] / 1e9 for g in ("fprop", "dgrad", "wgrad")},
+        "workload": "the same layer with MXFP4 operands (blocks of 32, UE8M0 scales, no tensor scale): X, W and "
+                    "dY each quantized in both forms (dY with SR), three kind::mxf4 GEMMs"}}
+    del f
+    lay = nv.LinearBF16(T_TOK, D_IN, D_OUT, device=dev)
+    bf_calls = [("fwd", lambda k: lay.fwd(x, w, y)), ("bwd", lambda k: lay.bwd(x, w, dy, dx, dw))]
+    per, ms = time_calls(bf_calls, args.steps, args.warmup, flush)
+    if nv.nvfp4_poll(ws) != 0 or nv.nvfp4_poll(lay.ws) != 0:
+        raise RuntimeError("device status in the MXFP4 / BF16 steps")
+    out["bf16_step"] = {
+        "value": FLOP_STEP / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms, "per_call_ms": per,
+        "fprop_tflops": FLOP_GEMM / per["fwd"] / 1e9,
+        "workload": "the same layer on the BF16 path: kind::f16 GEMMs with fp32 accumulation; the backward "
+                    "includes the bf16 transposes of W, dY and X (K-major operands)"}
+    del lay
+    torch.cuda.empty_cache()
+    return out
+
+
 def c1_latency(nv, dev) -> dict:
     """The 256 x 256 x 256 fprop of the small single-GEMM workload, reported as latency: the GEMM
     launch alone and the whole fprop (both quantize calls + GEMM), median over back-to-back
@@ -646,6 +713,10 @@ def main():
                     help="linear: the 8192x5120x20480 layer (the default line); ffn: the one-FFN step")
     ap.add_argument("--no-ffn", dest="ffn", action="store_false",
                     help="linear: skip the nested one-FFN step fields")
+    ap.add_argument("--no-c1", dest="c1", action="store_false",
+                    help="linear: skip the 256^3 fprop latency field")
+    ap.add_argument("--no-variants", dest="variants", action="store_false",
+                    help="linear: skip the nested MXFP4 and BF16 step fields")
     ap.add_argument("--ffn-fused-amax", action="store_true",
                     help="ffn: the GeLU kernels that also reduce their output's amax (slower as they stand)")
     args = ap.parse_args()
