@@ -62,18 +62,13 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(const uint4* __restrict__
 
 // ---------------------------------------------------------------------------------------
 // GeLU forward or backward with the amax of its bf16 output fused in (the amax pass of the
-// next quantize, which reads this output, is then skipped).  A CTA takes 16-row x 512-column
-// tiles of the [rows][cols] output:
-//   1. each thread computes four 16-byte chunks (8 elements of one row) with coalesced 16-byte
-//      loads and stores, reduces the plain magnitudes as packed bf16 integers, and stages the
-//      bf16 results in shared memory;
-//   2. each thread takes one column pair of the staged tile (16 rows x 2 columns, one 32-bit
-//      shared load per row), applies the 16-point RHT along the rows as f32x2 pairs and reduces
-//      the transformed magnitudes -- exactly what the amax pass computes from this output.
+// next quantize, which reads this output, is then skipped).  A thread owns a 16-row x 2-column
+// patch of the [rows][cols] output: 16 four-byte loads (a warp reads a full 128-byte line per
+// row), the GeLU of its 32 elements, 16 four-byte stores, then -- on the same registers -- the
+// packed-integer max of the bf16 magnitudes and the 16-point RHT of the column pair along the
+// rows (f32x2 pairs), exactly what the amax pass computes from this output.  No shared memory and
+// no barriers: the erfc/exp arithmetic dominates, and every warp stays busy with it.
 // ---------------------------------------------------------------------------------------
-constexpr int kGaRows = 16, kGaCols = 512, kGaThreads = 256;
-constexpr int kGaChunks = kGaRows * kGaCols / 8;   // 1024 sixteen-byte chunks per tile
-
 __device__ __forceinline__ uint32_t warp_max_u32_g(uint32_t v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -94,71 +89,42 @@ __device__ __forceinline__ void block_max_to(uint32_t v, uint32_t* dst, uint32_t
 }
 
 template <bool BWD>
-__device__ __forceinline__ uint4 gelu_chunk(const uint4 x, const uint4 d) {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    const uint32_t e[4] = {d.x, d.y, d.z, d.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        o[j] = BWD ? f32x2_to_bf16x2(bf16_lo(e[j]) * gelu_grad_f(bf16_lo(w[j])), bf16_hi(e[j]) * gelu_grad_f(bf16_hi(w[j])))
-                   : f32x2_to_bf16x2(gelu_f(bf16_lo(w[j])), gelu_f(bf16_hi(w[j])));
-    return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-template <bool BWD>
-__global__ void __launch_bounds__(kGaThreads, 4) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
-                                                            uint16_t* __restrict__ out, int64_t rows, int64_t cols,
-                                                            const SignMasks sm, uint32_t* __restrict__ amax_plain,
-                                                            uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
-    __shared__ __align__(16) uint16_t tile[kGaRows * kGaCols];
-    __shared__ uint32_t red[kGaThreads / 32];
-    const int tid = threadIdx.x;
-    const int64_t ntc = (cols + kGaCols - 1) / kGaCols;
-    const int64_t ntiles = (rows / kGaRows) * ntc;
+__global__ void __launch_bounds__(256, 4) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
+                                                        uint16_t* __restrict__ out, int64_t rows, int64_t cols,
+                                                        const SignMasks sm, uint32_t* __restrict__ amax_plain,
+                                                        uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
+    __shared__ uint32_t red[8];
+    const int64_t cpr = cols >> 1;
+    const int64_t groups = rows >> 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
     float mr = 0.0f;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int64_t tr = t / ntc, tc = t - tr * ntc;
-        const int64_t r0 = tr * kGaRows, c0 = tc * kGaCols;
-        // 1. GeLU of four chunks per thread: loads first, then compute, store and stage
-        uint4 x[kGaChunks / kGaThreads], d[kGaChunks / kGaThreads];
-        bool ok[kGaChunks / kGaThreads];
+    for (GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr); w.r < groups; w.next()) {
+        const int64_t base = (w.r << 4) * cols + (w.k << 1);
+        uint32_t x[16], d[16];
 #pragma unroll
-        for (int u = 0; u < kGaChunks / kGaThreads; ++u) {
-            const int j = tid + u * kGaThreads, i = j / (kGaCols / 8), ch = j % (kGaCols / 8);
-            const int64_t col = c0 + ch * 8;
-            ok[u] = col < cols;
-            const int64_t off = (r0 + i) * cols + col;
-            x[u] = ok[u] ? *reinterpret_cast<const uint4*>(h + off) : make_uint4(0, 0, 0, 0);
-            d[u] = (BWD && ok[u]) ? *reinterpret_cast<const uint4*>(dg + off) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 16; ++i) {
+            x[i] = *reinterpret_cast<const uint32_t*>(h + base + i * cols);
+            if (BWD) d[i] = *reinterpret_cast<const uint32_t*>(dg + base + i * cols);
         }
+        uint64_t f[16];
 #pragma unroll
-        for (int u = 0; u < kGaChunks / kGaThreads; ++u) {
-            const int j = tid + u * kGaThreads, i = j / (kGaCols / 8), ch = j % (kGaCols / 8);
-            const uint4 o = ok[u] ? gelu_chunk<BWD>(x[u], d[u]) : make_uint4(0, 0, 0, 0);
-            if (ok[u]) *reinterpret_cast<uint4*>(out + (r0 + i) * cols + c0 + ch * 8) = o;
-            *reinterpret_cast<uint4*>(tile + i * kGaCols + ch * 8) = o;
-            m = __vmaxu2(m, o.x & 0x7FFF7FFFu);
-            m = __vmaxu2(m, o.y & 0x7FFF7FFFu);
-            m = __vmaxu2(m, o.z & 0x7FFF7FFFu);
-            m = __vmaxu2(m, o.w & 0x7FFF7FFFu);
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t o = BWD ? f32x2_to_bf16x2(bf16_lo(d[i]) * gelu_grad_f(bf16_lo(x[i])),
+                                                     bf16_hi(d[i]) * gelu_grad_f(bf16_hi(x[i])))
+                                   : f32x2_to_bf16x2(gelu_f(bf16_lo(x[i])), gelu_f(bf16_hi(x[i])));
+            *reinterpret_cast<uint32_t*>(out + base + i * cols) = o;
+            m = __vmaxu2(m, o & 0x7FFF7FFFu);
+            f[i] = bf16x2_to_f2(o ^ sm.m[i]);
         }
-        __syncthreads();
-        // 2. the RHT amax of one column pair per thread (zero columns past `cols` add nothing)
-        {
-            uint64_t f[16];
+        rht16_pairs(f);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                f[i] = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(tile + i * kGaCols + 2 * tid) ^ sm.m[i]);
-            rht16_pairs(f);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float a, b;
-                f2_split(f[i], a, b);
-                mr = max3_abs(mr, a, b);
-            }
+        for (int i = 0; i < 16; i += 2) {
+            float a0, a1, b0, b1;
+            f2_split(f[i], a0, a1);
+            f2_split(f[i + 1], b0, b1);
+            mr = max3_abs(max3_abs(mr, a0, a1), b0, b1);
         }
-        __syncthreads();
     }
     const uint32_t mag = max(m & 0xFFFFu, m >> 16);
     if (mag >= 0x7F80u || !(mr < __int_as_float(0x7F800000))) atomicOr(flags, kFlagNonFinite);
@@ -249,19 +215,18 @@ cudaError_t launch_gelu_bwd(const uint16_t* h, const uint16_t* dg, uint16_t* dh,
 cudaError_t launch_gelu_amax(bool bwd, const uint16_t* h, const uint16_t* dg, uint16_t* out, int64_t rows,
                              int64_t cols, uint32_t signs, uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags,
                              cudaStream_t s) {
-    const int64_t tiles = (rows / kGaRows) * ((cols + kGaCols - 1) / kGaCols);
-    if (tiles == 0) return cudaSuccess;
+    const int64_t units = (rows >> 4) * (cols >> 1);
+    if (units == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = (int64_t)sms * 4;   // resident CTAs (16 KB of shared memory, <= 64 registers each)
-    const int grid = (int)(tiles < cap ? tiles : cap);
+    const int64_t want = (units + 255) / 256, cap = (int64_t)sms * 4;   // resident CTAs at <= 64 registers
+    const int grid = (int)(want < cap ? want : cap);
     if (bwd)
-        gelu_amax_kernel<true><<<grid, kGaThreads, 0, s>>>(h, dg, out, rows, cols, sign_masks(signs), amax_plain, amax_rht,
-                                                           flags);
+        gelu_amax_kernel<true><<<grid, 256, 0, s>>>(h, dg, out, rows, cols, sign_masks(signs), amax_plain, amax_rht, flags);
     else
-        gelu_amax_kernel<false><<<grid, kGaThreads, 0, s>>>(h, nullptr, out, rows, cols, sign_masks(signs), amax_plain,
-                                                            amax_rht, flags);
+        gelu_amax_kernel<false><<<grid, 256, 0, s>>>(h, nullptr, out, rows, cols, sign_masks(signs), amax_plain,
+                                                     amax_rht, flags);
     return cudaGetLastError();
 }
 

@@ -283,6 +283,28 @@ __device__ __forceinline__ void rht16_pairs(uint64_t (&v)[16]) {
     for (int j = 0; j < 16; ++j) v[j] = f2_mul(v[j], q);
 }
 
+// A grid-stride walk over the (row, chunk) grid of a [rows][chunks_per_row] tensor without a
+// division per step: the stride S = gridDim * blockDim is split once into whole rows and a
+// remainder, and the position advances by carry.
+struct GridWalk {
+    int64_t r, k;            // current (row, chunk)
+    int64_t dr, dk, cpr;     // stride in rows and chunks, chunks per row
+    __device__ __forceinline__ GridWalk(int64_t start, int64_t stride, int64_t cpr_) : cpr(cpr_) {
+        r = start / cpr;
+        k = start - r * cpr;
+        dr = stride / cpr;
+        dk = stride - dr * cpr;
+    }
+    __device__ __forceinline__ void next() {
+        r += dr;
+        k += dk;
+        if (k >= cpr) {
+            k -= cpr;
+            ++r;
+        }
+    }
+};
+
 // ---------------------------------------------------------------------------------------
 // Position of the scale of (form row r, K-block kb) in the 128x4-tile layout read by the
 // tcgen05 block-scaled MMA.

@@ -66,28 +66,6 @@ __device__ __forceinline__ void block_atomic_max(uint32_t v, uint32_t* dst, uint
     __syncthreads();
 }
 
-// A grid-stride walk over the (row, chunk) grid of a [rows][chunks_per_row] tensor without a
-// division per step: the stride S = gridDim * blockDim is split once into whole rows and a
-// remainder, and the position advances by carry.
-struct GridWalk {
-    int64_t r, k;            // current (row, chunk)
-    int64_t dr, dk, cpr;     // stride in rows and chunks, chunks per row
-    __device__ __forceinline__ GridWalk(int64_t start, int64_t stride, int64_t cpr_) : cpr(cpr_) {
-        r = start / cpr;
-        k = start - r * cpr;
-        dr = stride / cpr;
-        dk = stride - dr * cpr;
-    }
-    __device__ __forceinline__ void next() {
-        r += dr;
-        k += dk;
-        if (k >= cpr) {
-            k -= cpr;
-            ++r;
-        }
-    }
-};
-
 // ---------------------------------------------------------------------------------------
 // pass 1a: plain amax over a [rows][cols] bf16 tensor with leading dimension ld
 // ---------------------------------------------------------------------------------------
