@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
         // A warp covers two tile rows (16 blocks each); lanes 4a..4a+3 hold four consecutive
         // blocks of one row, whose scales leave as one 32-bit word.
         if (ROW) {
-#pragma unroll 1
+#pragma unroll
             for (int j = tid; j < kTileRows * (kTileCols / 16); j += kQuantThreads) {
                 const int r = j >> 4, b = j & 15;
                 const int64_t gr = r_base + r, gc = c_base + b * 16;
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
         // element are indexed by its position in the form, so each column's 16 elements are two
         // whole Philox calls.
         if (COL) {
-#pragma unroll 1
+#pragma unroll
             for (int j = tid; j < 4 * (kTileCols / 2); j += kQuantThreads) {
                 const int cp = j & (kTileCols / 2 - 1), g = j >> 7;   // a warp covers 64 columns of one group
                 const int c = 2 * cp;

@@ -58,6 +58,24 @@ def test_gelu_kernels_within_one_bf16_step(n):
             assert np.mean(d == 0) > 0.98, what
 
 
+def test_gelu_kernels_on_every_finite_bf16_input():
+    # every finite bf16 h (65280 values), forward and backward at three gradient scales: within
+    # one bf16 step of the exactly rounded fp64 values, and nearly all exact
+    m = nv()
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    bits = bits[np.isfinite(vals)]
+    h = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    got = _bits(m.nvfp4_gelu_fwd(to_device_bf16(h)))
+    d = _ulps(got, oracle.gelu_fwd(bits))
+    assert d.max() <= 1 and np.mean(d == 0) > 0.999, (int(d.max()), float(np.mean(d == 0)))
+    for scale in (1e-3, 1.0, 3e4):
+        dg = torch.full_like(h, scale)
+        got = _bits(m.nvfp4_gelu_bwd(to_device_bf16(h), to_device_bf16(dg)))
+        d = _ulps(got, oracle.gelu_bwd(bits, synth.bf16_bits(dg)))
+        assert d.max() <= 1 and np.mean(d == 0) > 0.999, (scale, int(d.max()), float(np.mean(d == 0)))
+
+
 @pytest.mark.parametrize("rows,cols", [(64, 256), (160, 512)])
 def test_gelu_amax_kernels(rows, cols):
     # the fused kernels' outputs stay within one bf16 step of the oracle, and the amax words they
