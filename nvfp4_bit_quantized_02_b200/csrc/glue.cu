@@ -19,9 +19,9 @@
 
 namespace nvfp4 {
 
-// Phi(h), the standard normal distribution function
-__device__ __forceinline__ float normal_cdf(float h) {
-    const float z = fabsf(h) * 0.70710678118654752f;
+// erfc(z) for z >= 0, times e^lnscale (the scale lets a caller keep the far tail, where erfc
+// falls below the normal fp32 range, at full precision)
+__device__ __forceinline__ float erfc_pos(float z, float lnscale) {
     const float t = __frcp_rn(fmaf(0.5f, z, 1.0f));
     float p = 0.17087277f;
     p = fmaf(t, p, -0.82215223f);
@@ -32,14 +32,30 @@ __device__ __forceinline__ float normal_cdf(float h) {
     p = fmaf(t, p, 0.09678418f);
     p = fmaf(t, p, 0.37409196f);
     p = fmaf(t, p, 1.00002368f);
-    const float erfc_z = t * expf(fmaf(-z, z, fmaf(t, p, -1.26551223f)));
-    return h >= 0.0f ? fmaf(-0.5f, erfc_z, 1.0f) : 0.5f * erfc_z;
+    return t * expf(fmaf(-z, z, fmaf(t, p, -1.26551223f)) + lnscale);
+}
+
+// Phi(h), the standard normal distribution function
+__device__ __forceinline__ float normal_cdf(float h) {
+    const float e = erfc_pos(fabsf(h) * 0.70710678118654752f, 0.0f);
+    return h >= 0.0f ? fmaf(-0.5f, e, 1.0f) : 0.5f * e;
 }
 
 __device__ __forceinline__ float gelu_f(float h) { return h * normal_cdf(h); }
 
-__device__ __forceinline__ float gelu_grad_f(float h) {
-    return fmaf(h, 0.39894228040143268f * expf(-0.5f * h * h), normal_cdf(h));
+// dg * GeLU'(h) = dg * (Phi(h) + h phi(h)).  Below h = -12 both terms fall towards the subnormal
+// fp32 range, where they would keep only a few significant bits that a large dg could lift back
+// into bf16's normal range: there they are evaluated scaled by 2^64 (inside the exponentials) and
+// the scale is undone after the product with dg.
+__device__ __forceinline__ float gelu_bwd_f(float h, float dg) {
+    const bool tail = h < -12.0f;
+    const float lnscale = tail ? 44.361419555836500f : 0.0f;   // 64 ln 2
+    const float z = fabsf(h) * 0.70710678118654752f;
+    const float e = erfc_pos(z, lnscale);
+    const float cdf = h >= 0.0f ? fmaf(-0.5f, e, 1.0f) : 0.5f * e;
+    const float pdf = 0.39894228040143268f * expf(fmaf(-0.5f * h, h, lnscale));
+    const float r = dg * fmaf(h, pdf, cdf);
+    return tail ? r * 5.42101086242752217e-20f : r;                // 2^-64
 }
 
 __global__ void __launch_bounds__(256) gelu_fwd_kernel(const uint4* __restrict__ h, uint4* __restrict__ g, int64_t n8,
@@ -71,13 +87,13 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(const uint4* __restrict__
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            o[j] = f32x2_to_bf16x2(bf16_lo(e[j]) * gelu_grad_f(bf16_lo(w[j])), bf16_hi(e[j]) * gelu_grad_f(bf16_hi(w[j])));
+            o[j] = f32x2_to_bf16x2(gelu_bwd_f(bf16_lo(w[j]), bf16_lo(e[j])), gelu_bwd_f(bf16_hi(w[j]), bf16_hi(e[j])));
         dh[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
         const float x = __uint_as_float((uint32_t)h_tail[threadIdx.x] << 16);
         const float y = __uint_as_float((uint32_t)dg_tail[threadIdx.x] << 16);
-        dh_tail[threadIdx.x] = (uint16_t)(f32x2_to_bf16x2(y * gelu_grad_f(x), 0.0f) & 0xFFFFu);
+        dh_tail[threadIdx.x] = (uint16_t)(f32x2_to_bf16x2(gelu_bwd_f(x, y), 0.0f) & 0xFFFFu);
     }
 }
 
@@ -131,8 +147,8 @@ __global__ void __launch_bounds__(256, 4) gelu_amax_kernel(const uint16_t* __res
         uint64_t f[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const uint32_t o = BWD ? f32x2_to_bf16x2(bf16_lo(d[i]) * gelu_grad_f(bf16_lo(x[i])),
-                                                     bf16_hi(d[i]) * gelu_grad_f(bf16_hi(x[i])))
+            const uint32_t o = BWD ? f32x2_to_bf16x2(gelu_bwd_f(bf16_lo(x[i]), bf16_lo(d[i])),
+                                                     gelu_bwd_f(bf16_hi(x[i]), bf16_hi(d[i])))
                                    : f32x2_to_bf16x2(gelu_f(bf16_lo(x[i])), gelu_f(bf16_hi(x[i])));
             *reinterpret_cast<uint32_t*>(out + base + i * cols) = o;
             m = __vmaxu2(m, o & 0x7FFF7FFFu);
