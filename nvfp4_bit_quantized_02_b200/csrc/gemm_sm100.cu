@@ -840,51 +840,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             const uint64_t adesc0 = desc_k_sw128(sbase), bdesc0 = desc_k_sw128(sbase + k2ABytes);
             int g = 0, local = 0;
             bool ok = true;
-            constexpr int tpb = OpFmt<F>::kTilesPerBlock;
-            // the scale tiles of stage g (K block kb of its tile) into TMEM scale slot g % k2SfRing
-            auto copy_scales = [&](int g_, int kb_) {
-                const int s_ = g_ % k2Stages, f_ = g_ % k2SfRing;
-                const int tiles = min(tpb, p.nkt - tpb * kb_);
-                const uint32_t t_sf = tmem + kSfCol0 + f_ * kSfColsPerStage;
-                const uint32_t sf_s = sbase + s_ * k2StageBytes + k2CodeBytes;
-#pragma unroll
-                for (int t = 0; t < tpb; ++t)
-                    if (t < tiles) {
-                        tmem_cp_sf_pair(t_sf + 4 * t, desc_sf(sf_s + 512 * t));
-                        tmem_cp_sf_pair(t_sf + 16 + 8 * t, desc_sf(sf_s + kSFABytes + 512 * t));
-                        tmem_cp_sf_pair(t_sf + 20 + 8 * t, desc_sf(sf_s + kSFABytes + tpb * 512 + 512 * t));
-                    }
-            };
             for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
-                // The first stage's scale copies go out before the accumulator is drained: they
-                // write the scale ring, not the accumulator, and the tensor pipe runs them in issue
-                // order behind the previous tile's MMAs, overlapping the epilogue's drain.
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait_cl(smem_u32(&full_bar[g % k2Stages]),
-                                                          (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns)))
-                    break;
-                tc_fence_after();
-                if (elect_one()) copy_scales(g, 0);
-                __syncwarp();
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait_cl(smem_u32(tempty_bar), ((uint32_t)local & 1u) ^ 1u, abort_flag,
                                                           p.flags, p.budget_ns)))
                     break;
                 tc_fence_after();
                 for (int kb = 0; kb < p.num_kb; ++kb, ++g) {
                     const int s = g % k2Stages, f = g % k2SfRing;
-                    if (kb > 0) {
-                        const bool landed = mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag,
-                                                         p.flags, p.budget_ns);
-                        if (!__all_sync(0xFFFFFFFFu, landed)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
+                    const bool landed =
+                        mbar_wait_cl(smem_u32(&full_bar[s]), (uint32_t)(g / k2Stages) & 1u, abort_flag, p.flags, p.budget_ns);
+                    if (!__all_sync(0xFFFFFFFFu, landed)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    constexpr int tpb = OpFmt<F>::kTilesPerBlock;
                     const int steps = min(4, p.kst - 4 * kb);
+                    const int tiles = min(tpb, p.nkt - tpb * kb);
                     const uint64_t aoff = (uint64_t)((s * k2StageBytes) >> 4);
                     const uint32_t t_sfa = tmem + kSfCol0 + f * kSfColsPerStage;
                     if (elect_one()) {
-                        if (kb > 0) copy_scales(g, kb);
+                        const uint32_t sf_s = sbase + s * k2StageBytes + k2CodeBytes;
+#pragma unroll
+                        for (int t = 0; t < tpb; ++t)
+                            if (t < tiles) {
+                                tmem_cp_sf_pair(t_sfa + 4 * t, desc_sf(sf_s + 512 * t));
+                                tmem_cp_sf_pair(t_sfa + 16 + 8 * t, desc_sf(sf_s + kSFABytes + 512 * t));
+                                tmem_cp_sf_pair(t_sfa + 20 + 8 * t, desc_sf(sf_s + kSFABytes + tpb * 512 + 512 * t));
+                            }
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             if (j < steps) {
