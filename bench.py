@@ -595,8 +595,10 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
 
 def c1_latency(nv, dev) -> dict:
     """The 256 x 256 x 256 fprop of the small single-GEMM workload, reported as latency: the GEMM
-    launch alone and the whole fprop (both quantize calls + GEMM), median over back-to-back
-    repetitions (the operands are L2-resident; a latency, not a bandwidth figure)."""
+    launch alone and the whole fprop (both quantize calls + GEMM), each as the median of 200
+    back-to-back calls from Python (host-bound at this size) and per call of a CUDA graph of 100
+    replayed five times (the device latency).  The operands are L2-resident: a latency, not a
+    bandwidth figure."""
     import synth
     x = synth.activations(256, 256, seed=0).to(dev)
     w = synth.weights(256, 256, seed=1).to(dev)
@@ -624,6 +626,31 @@ def c1_latency(nv, dev) -> dict:
             ts.append((a, b))
         torch.cuda.synchronize()
         res[name] = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        # the same calls captured once into a CUDA graph of 100 and replayed: the device-side
+        # latency without the host's per-call work (Python, argument checks, tensor-map encoding)
+        try:
+            s_cap = torch.cuda.Stream(dev)
+            s_cap.wait_stream(torch.cuda.current_stream(dev))
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s_cap):
+                with torch.cuda.graph(graph, stream=s_cap):
+                    for _ in range(100):
+                        fn()
+            torch.cuda.current_stream(dev).wait_stream(s_cap)
+            graph.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(5):
+                graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            res[name.replace("_us", "_graph_us")] = a.elapsed_time(b) * 1e3 / 500
+            del graph
+        except RuntimeError as e:   # a capture the runtime refused: report it, keep the line
+            torch.cuda.synchronize()
+            res[name.replace("_us", "_graph_us")] = None
+            res["graph_error"] = str(e)[:200]
     if nv.nvfp4_poll(ws) != 0:
         raise RuntimeError("device status in the small fprop")
     res["workload"] = "fprop 256x256x256: X N(0,1) 1x16 RNE, W N(0,0.02) 16x16 RNE, bf16 out"
