@@ -590,7 +590,32 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
                     "includes the bf16 transposes of W, dY and X (K-major operands)"}
     del lay
     torch.cuda.empty_cache()
+    out["wgrad_reduce_scatter"] = wgrad_reduce_scatter_fields(args, dev, flush, x, dy, dw)
     return out
+
+
+def wgrad_reduce_scatter_fields(args, dev, flush, x, dy, dw) -> dict:
+    """The wgrad GEMM (M = 20480, N = 5120, K = 8192 tokens) with its output stored (fp32), added
+    into 8 row shards of 2560 rows (the epilogue of the data-parallel reduce-scatter, here into
+    local buffers) and added into one fp32 buffer (gradient accumulation); each call timed alone
+    with L2 flushed before it."""
+    import nvfp4_bit_quantized_02_b200 as nv
+    ws = nv.Workspace(dev)
+    _, xc = nv.nvfp4_quantize_dual(x, mode=nv.RNE, rht_seed=3, ws=ws)
+    _, dyc = nv.nvfp4_quantize_dual(dy, mode=nv.SR, rht_seed=3, sr_seed=4, stream_row=1, stream_col=2, ws=ws)
+    share = D_OUT // 8
+    shards = [dw[o * share:(o + 1) * share] for o in range(8)]
+    res = {}
+    for name, fn in (("stored", lambda k: nv.nvfp4_gemm(dyc, xc, out=dw, ws=ws)),
+                     ("8 owners", lambda k: nv.nvfp4_gemm_reduce_scatter(dyc, xc, shards, share, ws=ws)),
+                     ("1 owner", lambda k: nv.nvfp4_gemm_reduce_scatter(dyc, xc, [dw], D_OUT, ws=ws))):
+        per, _ = time_calls([(name, fn)], args.steps, args.warmup, flush)
+        res[name] = per[name]
+    if nv.nvfp4_poll(ws) != 0:
+        raise RuntimeError("device status in the wgrad reduce-scatter timing")
+    return {"ms": res, "tflops": {k: FLOP_GEMM / v / 1e9 for k, v in res.items()},
+            "workload": "the layer's wgrad GEMM, fp32 output stored, reduce-added into 8 local row shards, and "
+                        "reduce-added into one buffer"}
 
 
 def c1_latency(nv, dev) -> dict:

@@ -185,6 +185,28 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, i
                         nvfp4_dtype out_dtype, void* ws, nvfp4_stream_t stream);
 
 /*
+ * The same product as nvfp4_gemm with fp32 output, ADDED into row shards instead of stored: the
+ * data-parallel weight gradient (gist.science 2.B: dW is a sum over tokens, so each replica holds a
+ * K-partial that the replicas sum), reduced as the GEMM's epilogue writes it.  Owner o receives
+ * rows [o * owner_rows, min(M, (o + 1) * owner_rows)) of D: shards[o][r][c] += D[o * owner_rows + r][c],
+ * row stride ldd (elements).  shards is a HOST array of n_owners device addresses valid on the
+ * calling device (local buffers, or other GPUs' buffers through peer mappings); each output tile
+ * is added by the TMA engine (an fp32 bulk tensor reduce-add) once, so a shard accumulates whatever
+ * it held before: zero it for a plain reduce-scatter, or pass one owner (owner_rows >= M) to
+ * accumulate a gradient into an existing fp32 buffer.  Every add of the call is complete in memory
+ * when the call's work on `stream` is complete; the caller orders the shards' later readers (a
+ * stream event, or a collective as a barrier between GPUs).  Adds from several calls into one
+ * shard at the same time are per-element reductions in an order that is not fixed, so their sum
+ * is reproducible only up to fp32 rounding order.  Shape rules: those of nvfp4_gemm;
+ * 1 <= n_owners <= 8; owner_rows % 32 == 0 and n_owners == ceil(M / owner_rows); shards 16-byte
+ * aligned; ldd * 4 % 16 == 0 (NVFP4_ERR_SHAPE / NVFP4_ERR_ALIGN / NVFP4_ERR_NULL otherwise,
+ * before any device work).
+ */
+nvfp4_status nvfp4_gemm_reduce_scatter(const nvfp4_tensor* a, const nvfp4_tensor* b, float* const* shards,
+                                       int n_owners, int64_t owner_rows, int64_t ldd, void* ws,
+                                       nvfp4_stream_t stream);
+
+/*
  * Linear layer y = x w^T with NVFP4 GEMMs (gist.science 2.B): all buffers caller-owned.
  *   xq      [T][d]   1x16 RNE           (fprop A)
  *   xq_rht  [d][T]   RHT 1x16 RNE       (wgrad B)

@@ -81,6 +81,7 @@ def _lib():
             "nvfp4_quantize_dual_shard": ([vp, i64, i64, i64, i64, i64, i32, u64, u64, u32, u32, T, T, vp, vp], i32),
             "nvfp4_transpose_2d": ([T, T, vp], i32),
             "nvfp4_gemm": ([T, T, vp, i64, i32, vp, vp], i32),
+            "nvfp4_gemm_reduce_scatter": ([T, T, c.POINTER(vp), i32, i64, i64, vp, vp], i32),
             "nvfp4_linear_fwd": ([vp, vp, vp, c.POINTER(CLinearCtx), vp], i32),
             "nvfp4_linear_bwd": ([vp, u64, vp, vp, c.POINTER(CLinearCtx), vp], i32),
             "nvfp4_gelu_fwd": ([vp, vp, i64, vp], i32),
@@ -275,11 +276,12 @@ def nvfp4_quantize_dual_dp(x: torch.Tensor, group, row_offset: int, rows_total: 
                            ws: Workspace | None = None, stream=None):
     """Both forms of this rank's token shard, equal to the slices of the whole batch's forms: the
     shard amax, a MAX all-reduce of the two amax words over ``group`` (torch.distributed), then
-    the shard's pass 2."""
+    the shard's pass 2.  Without an initialized process group there is one rank, whose shard is
+    the batch, and no exchange."""
     import torch.distributed as dist
     ws = nvfp4_amax(x, True, rht_seed, ws, stream)
-    words = ws.amax_words()
-    dist.all_reduce(words, op=dist.ReduceOp.MAX, group=group)
+    if dist.is_initialized():
+        dist.all_reduce(ws.amax_words(), op=dist.ReduceOp.MAX, group=group)
     return nvfp4_quantize_dual_shard(x, row_offset, rows_total, mode, rht_seed, sr_seed, stream_row, stream_col,
                                      out_row, out_col, ws, stream)
 
@@ -320,6 +322,32 @@ def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=torch.bfloat16, out: to
     st = _lib().nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), out.stride(0), code, ws.ptr, _stream(stream))
     _check(st, "nvfp4_gemm")
     return out
+
+
+def nvfp4_gemm_reduce_scatter(a: NVFP4Tensor, b: NVFP4Tensor, shards, owner_rows: int,
+                              ws: Workspace | None = None, stream=None) -> None:
+    """shards[o] += rows [o*owner_rows, (o+1)*owner_rows) of s_tA s_tB * A . B^T (fp32 adds).
+
+    shards: fp32 [rows_o][N] tensors with one row stride (local, or another GPU's buffer through
+    a peer mapping). One owner with owner_rows >= rows accumulates the whole product into it.
+    """
+    if not shards:
+        raise ValueError("nvfp4_gemm_reduce_scatter needs at least one shard")
+    ld = shards[0].stride(0)
+    for t in shards:
+        if t.dtype != torch.float32 or t.dim() != 2 or t.stride(1) != 1 or t.stride(0) != ld:
+            raise ValueError("shards must be fp32 2-D row-major tensors with one row stride")
+        if t.shape[1] != b.rows:
+            raise ValueError("each shard has N = b.rows columns")
+    for o, t in enumerate(shards):
+        if t.shape[0] < min(owner_rows, a.rows - o * owner_rows):
+            raise ValueError(f"shard {o} holds fewer rows than its owner's share")
+    addrs = (ctypes.c_void_p * len(shards))(*[t.data_ptr() for t in shards])
+    ws = ws or default_workspace()
+    ca, cb = a.c(), b.c()
+    st = _lib().nvfp4_gemm_reduce_scatter(ctypes.byref(ca), ctypes.byref(cb), addrs, len(shards), owner_rows, ld,
+                                          ws.ptr, _stream(stream))
+    _check(st, "nvfp4_gemm_reduce_scatter")
 
 
 def nvfp4_gelu_fwd(h: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -528,20 +556,53 @@ class DPLinear:
     - W: quantized on every rank from the same replica (identical forms, no exchange).
     - dW: each rank's wgrad GEMM gives the partial sum over its tokens; the partials are
       reduce-scattered (fp32 sum) over the group, each rank keeping rows dp_dw_rows(n, rank,
-      world).  The wgrad GEMM runs first and the reduce-scatter overlaps the dgrad GEMM.
+      world).  dw_reduce="nccl": the wgrad GEMM stores the partial, and an NCCL reduce-scatter
+      overlaps the dgrad GEMM.  dw_reduce="fused": the wgrad GEMM's epilogue adds each output
+      tile into its owner's shard directly (nvfp4_gemm_reduce_scatter into the ranks' symmetric
+      buffers, through peer addresses), so the exchange runs inside the GEMM; a 4-byte all-reduce
+      after the dgrad GEMM is the barrier that orders every rank's adds before the owner reads
+      its shard.  Two shard buffers alternate between steps, so a buffer is zeroed one whole
+      step (one barrier) before any rank adds into it again.
     """
 
-    def __init__(self, T: int, d: int, n: int, group=None, rht_seed: int = 0, device=None):
+    def __init__(self, T: int, d: int, n: int, group=None, rht_seed: int = 0, device=None,
+                 dw_reduce: str = "nccl"):
         import torch.distributed as dist
+        if dw_reduce not in ("nccl", "fused"):
+            raise ValueError("dw_reduce is 'nccl' or 'fused'")
         self.group = group
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self.T, self.d, self.n, self.rht_seed = T, d, n, rht_seed
         self.ctx = LinearContext(T, d, n, rht_seed=rht_seed, device=device)
-        self.dw_partial = torch.empty((n, d), dtype=torch.float32, device=device)
         r0, r1 = dp_dw_rows(n, self.rank, self.world)
         self.dw = torch.empty((r1 - r0, d), dtype=torch.float32, device=device)
+        self.dw_reduce = dw_reduce
+        if dw_reduce == "nccl":
+            self.dw_partial = torch.empty((n, d), dtype=torch.float32, device=device)
+            return
+        per = r1 - r0
+        if per % 32 or self.world > 8:
+            raise ValueError("the fused reduce-scatter needs n / world % 32 == 0 and at most 8 ranks")
+        self._rs_bufs, self._rs_peers, self._rs_step = [], [], 0
+        for _ in range(2):
+            if dist.is_initialized():
+                import torch.distributed._symmetric_memory as symm_mem
+                buf = symm_mem.empty((per, d), dtype=torch.float32, device=device)
+                buf.zero_()
+                h = symm_mem.rendezvous(buf, group if group is not None else dist.group.WORLD)
+                peers = [buf if p == self.rank else h.get_buffer(p, (per, d), torch.float32)
+                         for p in range(self.world)]
+            else:
+                buf = torch.zeros((per, d), dtype=torch.float32, device=device)
+                peers = [buf]
+            self._rs_bufs.append(buf)
+            self._rs_peers.append(peers)
+        self._rs_flag = torch.zeros(1, dtype=torch.float32, device=device)
+        if dist.is_initialized():
+            torch.cuda.synchronize(device)
+            dist.barrier(group)   # every shard is zero before any rank adds into it
 
     def fwd(self, x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
         c = self.ctx
@@ -559,6 +620,16 @@ class DPLinear:
         nvfp4_quantize_dual_dp(dy, self.group, off, total, mode=SR, rht_seed=self.rht_seed, sr_seed=sr_seed,
                                stream_row=STREAM_DGRAD, stream_col=STREAM_WGRAD, out_row=c.dyq, out_col=c.dyq_rht,
                                ws=c.ws)
+        if self.dw_reduce == "fused":
+            j = self._rs_step & 1
+            self._rs_step += 1
+            nvfp4_gemm_reduce_scatter(c.dyq_rht, c.xq_rht, self._rs_peers[j], self.dw.shape[0], ws=c.ws)
+            dx = nvfp4_gemm(c.dyq, c.wqt, out=dx, ws=c.ws)
+            if dist.is_initialized():
+                dist.all_reduce(self._rs_flag, group=self.group)   # every rank's adds are complete
+            self.dw.copy_(self._rs_bufs[j])
+            self._rs_bufs[j].zero_()
+            return dx
         nvfp4_gemm(c.dyq_rht, c.xq_rht, out=self.dw_partial, ws=c.ws)
         work = None
         if self.world > 1:

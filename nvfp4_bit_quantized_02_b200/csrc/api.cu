@@ -391,6 +391,32 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, i
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_gemm_reduce_scatter(const nvfp4_tensor* a, const nvfp4_tensor* b, float* const* shards,
+                                       int n_owners, int64_t owner_rows, int64_t ldd, void* ws,
+                                       nvfp4_stream_t stream) {
+    if (!a || !b || !shards) return NVFP4_ERR_NULL;
+    if (nvfp4_status st = check_form_buffers(a, false)) return st;
+    if (nvfp4_status st = check_form_buffers(b, false)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    const int64_t M = a->rows, N = b->rows, K = a->k;
+    if (b->k != K) return NVFP4_ERR_ARG;
+    if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return NVFP4_ERR_LIMIT;
+    if (n_owners < 1 || n_owners > 8 || owner_rows < 32 || owner_rows % 32 != 0) return NVFP4_ERR_SHAPE;
+    if ((M + owner_rows - 1) / owner_rows != n_owners) return NVFP4_ERR_SHAPE;
+    if (ldd < N) return NVFP4_ERR_SHAPE;
+    if ((ldd * 4) % 16 != 0) return NVFP4_ERR_ALIGN;
+    for (int o = 0; o < n_owners; ++o) {
+        if (!shards[o]) return NVFP4_ERR_NULL;
+        if (!aligned16(shards[o])) return NVFP4_ERR_ALIGN;
+    }
+    if (nvfp4_status st = check_device()) return st;
+    return from_cuda(launch_gemm_nvf4_reduce_scatter(a->codes, a->scales, a->tensor_scale, M, b->codes, b->scales,
+                                                     b->tensor_scale, N, K, shards, n_owners, owner_rows, ldd,
+                                                     &ws_of(ws)->flags, g_budget_ns.load(),
+                                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
 static nvfp4_status check_ctx(const nvfp4_linear_ctx* c) {
     if (!c) return NVFP4_ERR_NULL;
     if (c->T <= 0 || c->d <= 0 || c->n <= 0) return NVFP4_ERR_SHAPE;

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
@@ -247,6 +248,14 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  "r"(src), "r"(x), "r"(y)
                  : "memory");
 }
+// shared -> global tile reduce-add by the TMA (fp32 add into the destination), in this thread's
+// bulk group
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -273,6 +282,17 @@ struct GemmParams {
     int32_t group_n;        // raster: 1 = groups of kGroup N tiles sweep all M tiles, 0 = the transpose
     uint32_t* flags;
     uint64_t budget_ns;
+    // reduce-scatter epilogue (0 owners: plain stores to D): output rows [o * owner_rows,
+    // (o + 1) * owner_rows) are added into owner o's shard through its own tensor map
+    int32_t n_owners;
+    int32_t owner_rows;
+};
+
+// The shards of a reduce-scatter epilogue: one fp32 output map per owner (a local buffer or
+// another GPU's, through its peer address)
+constexpr int kMaxOwners = 8;
+struct OwnerMaps {
+    CUtensorMap m[kMaxOwners];
 };
 
 constexpr int kEpi1Warps = 16;                     // four warps per TMEM lane quadrant, 64 columns each
@@ -309,10 +329,12 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm,
 // has been read by its store; the last boxes of a tile hand over to the first ones of the next.
 // One mbarrier per box position keeps every waiting warp at most one phase ahead of it.  Returns
 // false on abort.
+// With owner maps (the reduce-scatter epilogue) each box is added into the shard of the owner of
+// its rows instead of stored.
 template <int kSlots>
-__device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, uint8_t* store_area, uint64_t* boxgo_bar,
-                                            const uint32_t (&r)[2][32], int ew, int local, int x0, int y,
-                                            const GemmParams& p, float alpha, volatile uint32_t* abort_flag) {
+__device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtensorMap* owner_maps, uint8_t* store_area,
+                                            uint64_t* boxgo_bar, const uint32_t (&r)[2][32], int ew, int local, int x0,
+                                            int y, const GemmParams& p, float alpha, volatile uint32_t* abort_flag) {
     const int lane = threadIdx.x & 31;
     const int nbox = p.out_fp32 ? 2 : 1;
     const int nb = kEpi1Warps * nbox;   // boxes per tile, a multiple of kSlots
@@ -356,7 +378,14 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, uint8_t* sto
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-            if (x < p.N && y < p.M) tma_store_2d(tmD, sbase, x, y);
+            if (x < p.N && y < p.M) {
+                if (owner_maps) {
+                    const int o = y / p.owner_rows;
+                    tma_reduce_add_2d(&owner_maps[o], sbase, x, y - o * p.owner_rows);
+                } else {
+                    tma_store_2d(tmD, sbase, x, y);
+                }
+            }
             bulk_commit();
             bulk_wait_read_all();
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&boxgo_bar[(b + kSlots) % nb])) : "memory");
@@ -369,7 +398,7 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, uint8_t* sto
 template <bool MX>
 __global__ void __launch_bounds__(kGemm1Threads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmD, GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmD, const __grid_constant__ OwnerMaps om, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* store_area = smem + kStages * kStageBytes;
@@ -538,7 +567,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
-            ok = store_boxes<kStoreSlots>(&tmD, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64, tm * kBM + q * 32,
+            ok = store_boxes<kStoreSlots>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64, tm * kBM + q * 32,
                                           p, alpha, abort_flag);
         }
         if (lane == 0) bulk_wait_all();   // this lane's stores are in global memory before the CTA exits
@@ -750,7 +779,7 @@ template <int F>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                         const __grid_constant__ CUtensorMap tmD, GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmD, const __grid_constant__ OwnerMaps om, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* store_area = smem + k2Stages * k2StageBytes;
@@ -932,7 +961,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(drained) : "memory");
-            ok = store_boxes<k2StoreSlots>(&tmD, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
+            ok = store_boxes<k2StoreSlots>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
                                            tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag);
         }
         if (lane == 0) bulk_wait_all();
@@ -1056,11 +1085,36 @@ static int sm_count() {
     return n;
 }
 
+// Output maps of the reduce-scatter epilogue: owner o's shard holds rows
+// [o * owner_rows, min(M, (o + 1) * owner_rows)) of D, fp32, row stride ldd
+static bool make_owner_maps(OwnerMaps* om, float* const* shards, int n_owners, int64_t owner_rows, int64_t M, int64_t N,
+                            int64_t ldd) {
+    *om = OwnerMaps{};
+    for (int o = 0; o < n_owners; ++o) {
+        const int64_t rows = std::min(owner_rows, M - o * owner_rows);
+        if (rows < 1 || !make_out_map(&om->m[o], shards[o], rows, N, ldd, true)) return false;
+    }
+    return true;
+}
+
+// n_owners > 0: the reduce-scatter epilogue (fp32 adds into owner_d[o]) replaces the stores to d
 template <bool MX>
 static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
                                const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                                void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, float* const* owner_d = nullptr, int n_owners = 0,
+                               int64_t owner_rows = 0) {
+    if (n_owners < 0 || n_owners > kMaxOwners || (n_owners > 0 && (!out_fp32 || owner_rows < 32 || owner_rows % 32 != 0 ||
+                                                                   (M + owner_rows - 1) / owner_rows != n_owners)))
+        return cudaErrorInvalidValue;
+    static const OwnerMaps no_owners{};
+    OwnerMaps om_local;
+    const OwnerMaps* om = &no_owners;
+    if (n_owners > 0) {
+        if (!make_owner_maps(&om_local, owner_d, n_owners, owner_rows, M, N, ldd)) return cudaErrorInvalidValue;
+        om = &om_local;
+        d = owner_d[0];   // the plain output map is built but never written
+    }
     GemmParams p;
     p.sfa = a_scales;
     p.sfb = b_scales;
@@ -1082,6 +1136,8 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     p.group_n = (M <= N) ? 1 : 0;   // operands are M x K and N x K: sweep the smaller one
     p.flags = flags;
     p.budget_ns = budget_ns;
+    p.n_owners = n_owners;
+    p.owner_rows = (int32_t)owner_rows;
     const int sms = sm_count();
     // SM-pair tiles for M >= 256 (fewer operand bytes per SM per K block, a deeper ring);
     // NVFP4_GEMM_VARIANT=1sm selects the 1-SM kernel for every shape (read on every call)
@@ -1101,7 +1157,8 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         if (!make_out_map(&td2, d, M, N, ldd, out_fp32) || !make_sf_map(&tsa, a_scales, p.sfa_row_tiles, p.nkt, 1, sfe) ||
             !make_sf_map(&tsb, b_scales, p.sfb_row_tiles, p.nkt, 2, sfe))
             return cudaErrorInvalidValue;
-        gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2, p);
+        gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2,
+                                                                                                      *om, p);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> attr_1sm{0};
@@ -1113,7 +1170,7 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     CUtensorMap td;
     if (!make_out_map(&td, d, M, N, ldd, out_fp32)) return cudaErrorInvalidValue;
-    gemm_nvf4_kernel<MX><<<grid, kGemm1Threads, kGemmSmem, stream>>>(ta, tb, td, p);
+    gemm_nvf4_kernel<MX><<<grid, kGemm1Threads, kGemmSmem, stream>>>(ta, tb, td, *om, p);
     return cudaGetLastError();
 }
 
@@ -1123,6 +1180,14 @@ cudaError_t launch_gemm_nvf4(const uint8_t* a_codes, const uint8_t* a_scales, co
                              cudaStream_t stream) {
     return launch_gemm<false>(a_codes, a_scales, a_st, M, b_codes, b_scales, b_st, N, K, d, ldd, out_fp32, flags,
                               budget_ns, stream);
+}
+
+cudaError_t launch_gemm_nvf4_reduce_scatter(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
+                                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N,
+                                            int64_t K, float* const* shards, int n_owners, int64_t owner_rows, int64_t ldd,
+                                            uint32_t* flags, uint64_t budget_ns, cudaStream_t stream) {
+    return launch_gemm<false>(a_codes, a_scales, a_st, M, b_codes, b_scales, b_st, N, K, nullptr, ldd, true, flags,
+                              budget_ns, stream, shards, n_owners, owner_rows);
 }
 
 // MXFP4 operands carry no tensor scale (null scale pointers: the epilogue's factor is 1)
@@ -1180,7 +1245,8 @@ cudaError_t launch_gemm_bf16(const uint16_t* a, int64_t lda, const uint16_t* b, 
     const int64_t ntiles = (int64_t)p.tiles_m * p.tiles_n;
     const int64_t pairs = ntiles < sms / 2 ? ntiles : sms / 2;
     // the scale maps are not read by the bf16 instantiation; valid maps are passed in their place
-    gemm_nvf4_2sm_kernel<kBF16><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta, tb, ta, tb, td, p);
+    static const OwnerMaps no_owners{};
+    gemm_nvf4_2sm_kernel<kBF16><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta, tb, ta, tb, td, no_owners, p);
     return cudaGetLastError();
 }
 
