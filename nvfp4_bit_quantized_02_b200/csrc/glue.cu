@@ -5,10 +5,16 @@
 //   dh = dg * (Phi(h) + h * phi(h)),  phi = N(0,1) density.
 // Phi comes from erfc(|h| / sqrt 2) through the Chebyshev fit of erfc(z) exp(z^2) in
 // t = 1 / (1 + z/2) published by Press, Teukolsky, Vetterling and Flannery (Numerical Recipes,
-// 2nd ed., section 6.2), whose fractional error is below 1.2e-7 for every z >= 0; evaluated with
-// fp32 FMAs it stays within a few 1e-7, far inside the half-step of the bf16 results (the tests
-// sweep every finite bf16 input against the fp64 oracle).  The library erfcf took about three
-// times the instructions and made these kernels compute-bound.
+// 2nd ed., section 6.2), whose fractional error is below 1.2e-7 for every z >= 0.
+// Two evaluations:
+//   - pairs (|h| <= 12, the bulk): two elements per f32x2 instruction, t from the approximate
+//     reciprocal and e^x as 2^(x log2 e) on the multi-function unit.  The fp32 rounding of the
+//     exponent's argument (|x| up to ~75 at |h| = 12) dominates the error: relative ~1e-5 at the
+//     far end, ~1e-6 for |h| < 3, against the bf16 results' half-step of 2^-9;
+//   - scalar (|h| > 12, inf, NaN): IEEE reciprocal and expf, with the far tail scaled (below).
+// The tests sweep every finite bf16 input against the fp64 oracle (within one bf16 step, more
+// than 99.9 % exact).  The library erfcf took about three times the instructions and made these
+// kernels compute-bound; the pair form streams at about the speed of a copy.
 // Elementwise kernels: 16-byte loads and stores, grid-stride.
 #include <cuda_runtime.h>
 
@@ -43,6 +49,78 @@ __device__ __forceinline__ float normal_cdf(float h) {
 
 __device__ __forceinline__ float gelu_f(float h) { return h * normal_cdf(h); }
 
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2c(float v) { return f2(v, v); }
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+// e^x for a pair, x >= -80 (normal results)
+__device__ __forceinline__ uint64_t exp_pair(uint64_t x) {
+    float a, b;
+    f2_split(f2_mul(x, f2c(1.4426950408889634f)), a, b);
+    return f2(ex2_approx(a), ex2_approx(b));
+}
+// erfc(|h| / sqrt 2) of a pair with |h| <= 12, and m2 = -h^2 / 2 (exact: h is a bf16 value)
+__device__ __forceinline__ uint64_t erfc_pair(float hl, float hh, uint64_t& m2) {
+    const float dl = fmaf(fabsf(hl), 0.35355339059327376f, 1.0f), dh = fmaf(fabsf(hh), 0.35355339059327376f, 1.0f);
+    const uint64_t t = f2(rcp_approx(dl), rcp_approx(dh));   // 1 / (1 + z/2)
+    uint64_t p = f2c(0.17087277f);
+    p = f2_fma(t, p, f2c(-0.82215223f));
+    p = f2_fma(t, p, f2c(1.48851587f));
+    p = f2_fma(t, p, f2c(-1.13520398f));
+    p = f2_fma(t, p, f2c(0.27886807f));
+    p = f2_fma(t, p, f2c(-0.18628806f));
+    p = f2_fma(t, p, f2c(0.09678418f));
+    p = f2_fma(t, p, f2c(0.37409196f));
+    p = f2_fma(t, p, f2c(1.00002368f));
+    const uint64_t h2 = f2(hl, hh);
+    m2 = f2_mul(f2_mul(h2, f2c(-0.5f)), h2);
+    return f2_mul(t, exp_pair(f2_add(f2_fma(t, p, f2c(-1.26551223f)), m2)));
+}
+// GeLU of a bf16 pair (|h| <= 12): h Phi(h) = max(h, 0) - |h| erfc(|h| / sqrt 2) / 2
+__device__ __forceinline__ uint32_t gelu_pair(uint32_t w) {
+    const float hl = bf16_lo(w), hh = bf16_hi(w);
+    uint64_t m2;
+    const uint64_t e = erfc_pair(hl, hh, m2);
+    float gl, gh;
+    f2_split(f2_fma(f2(fabsf(hl) * -0.5f, fabsf(hh) * -0.5f), e, f2(fmaxf(hl, 0.0f), fmaxf(hh, 0.0f))), gl, gh);
+    return f32x2_to_bf16x2(gl, gh);
+}
+// dg GeLU'(h) of a bf16 pair (|h| <= 12): Phi(h) = [h >= 0] -+ erfc / 2, phi(h) = e^(-h^2/2) / sqrt(2 pi)
+__device__ __forceinline__ uint32_t gelu_bwd_pair(uint32_t w, uint32_t d) {
+    const float hl = bf16_lo(w), hh = bf16_hi(w);
+    uint64_t m2;
+    const uint64_t e = erfc_pair(hl, hh, m2);
+    const uint64_t cdf = f2_fma(f2(hl >= 0.0f ? -0.5f : 0.5f, hh >= 0.0f ? -0.5f : 0.5f), e,
+                                f2(hl >= 0.0f ? 1.0f : 0.0f, hh >= 0.0f ? 1.0f : 0.0f));
+    const uint64_t hc = f2_mul(f2(hl, hh), f2c(0.39894228040143268f));
+    float rl, rh;
+    f2_split(f2_mul(f2_fma(hc, exp_pair(m2), cdf), bf16x2_to_f2(d)), rl, rh);
+    return f32x2_to_bf16x2(rl, rh);
+}
+// a bf16 pair whose magnitudes are both <= 12 (neither inf nor NaN)
+__device__ __forceinline__ bool pair_in_range(uint32_t w) {
+    return __vcmpleu2(w & 0x7FFF7FFFu, 0x41404140u) == 0xFFFFFFFFu;
+}
+__device__ __forceinline__ bool quad_in_range(const uint4& v) {
+    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16) <= 0x4140u;
+}
+__device__ __forceinline__ uint32_t gelu_word(uint32_t w) {
+    return pair_in_range(w) ? gelu_pair(w) : f32x2_to_bf16x2(gelu_f(bf16_lo(w)), gelu_f(bf16_hi(w)));
+}
+
 // dg * GeLU'(h) = dg * (Phi(h) + h phi(h)).  Below h = -12 both terms fall towards the subnormal
 // fp32 range, where they would keep only a few significant bits that a large dg could lift back
 // into bf16's normal range: there they are evaluated scaled by 2^64 (inside the exponentials) and
@@ -58,6 +136,11 @@ __device__ __forceinline__ float gelu_bwd_f(float h, float dg) {
     return tail ? r * 5.42101086242752217e-20f : r;                // 2^-64
 }
 
+__device__ __forceinline__ uint32_t gelu_bwd_word(uint32_t w, uint32_t d) {
+    return pair_in_range(w) ? gelu_bwd_pair(w, d)
+                            : f32x2_to_bf16x2(gelu_bwd_f(bf16_lo(w), bf16_lo(d)), gelu_bwd_f(bf16_hi(w), bf16_hi(d)));
+}
+
 __global__ void __launch_bounds__(256) gelu_fwd_kernel(const uint4* __restrict__ h, uint4* __restrict__ g, int64_t n8,
                                                        const uint16_t* __restrict__ h_tail, uint16_t* __restrict__ g_tail,
                                                        int tail) {
@@ -65,8 +148,13 @@ __global__ void __launch_bounds__(256) gelu_fwd_kernel(const uint4* __restrict__
         const uint4 v = h[i];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
+        if (quad_in_range(v)) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = f32x2_to_bf16x2(gelu_f(bf16_lo(w[j])), gelu_f(bf16_hi(w[j])));
+            for (int j = 0; j < 4; ++j) o[j] = gelu_pair(w[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = gelu_word(w[j]);
+        }
         g[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
@@ -85,9 +173,13 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(const uint4* __restrict__
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         const uint32_t e[4] = {d.x, d.y, d.z, d.w};
         uint32_t o[4];
+        if (quad_in_range(v)) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            o[j] = f32x2_to_bf16x2(gelu_bwd_f(bf16_lo(w[j]), bf16_lo(e[j])), gelu_bwd_f(bf16_hi(w[j]), bf16_hi(e[j])));
+            for (int j = 0; j < 4; ++j) o[j] = gelu_bwd_pair(w[j], e[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = gelu_bwd_word(w[j], e[j]);
+        }
         dh[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (blockIdx.x == 0 && (int)threadIdx.x < tail) {
@@ -99,12 +191,15 @@ __global__ void __launch_bounds__(256) gelu_bwd_kernel(const uint4* __restrict__
 
 // ---------------------------------------------------------------------------------------
 // GeLU forward or backward with the amax of its bf16 output fused in (the amax pass of the
-// next quantize, which reads this output, is then skipped).  A thread owns a 16-row x 2-column
-// patch of the [rows][cols] output: 16 four-byte loads (a warp reads a full 128-byte line per
-// row), the GeLU of its 32 elements, 16 four-byte stores, then -- on the same registers -- the
-// packed-integer max of the bf16 magnitudes and the 16-point RHT of the column pair along the
-// rows (f32x2 pairs), exactly what the amax pass computes from this output.  No shared memory and
-// no barriers: the erfc/exp arithmetic dominates, and every warp stays busy with it.
+// next quantize, which reads this output, is then skipped).  A CTA walks 32-row x 256-column
+// tiles of the [rows][cols] output:
+//   1. each thread streams four 16-byte chunks of the tile (the plain kernel's access pattern),
+//      stores their GeLU to global memory and to a shared-memory copy of the tile, and keeps the
+//      packed-integer max of the bf16 magnitudes;
+//   2. after a barrier each thread takes one column pair of one 16-row group from shared memory
+//      (a warp reads 32 consecutive words of a row: no bank conflicts) and applies the 16-point
+//      RHT along the rows to it (f32x2 pairs), keeping the max magnitude -- exactly what the amax
+//      pass computes from this output.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t warp_max_u32_g(uint32_t v) {
 #pragma unroll
@@ -125,43 +220,81 @@ __device__ __forceinline__ void block_max_to(uint32_t v, uint32_t* dst, uint32_t
     __syncthreads();
 }
 
+constexpr int kGaRows = 32, kGaWords = 128;   // a tile: 32 rows x 256 bf16 (128 words a row)
+
 template <bool BWD>
-__global__ void __launch_bounds__(256, 4) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
+__global__ void __launch_bounds__(256) gelu_amax_kernel(const uint16_t* __restrict__ h, const uint16_t* __restrict__ dg,
                                                         uint16_t* __restrict__ out, int64_t rows, int64_t cols,
                                                         const SignMasks sm, uint32_t* __restrict__ amax_plain,
                                                         uint32_t* __restrict__ amax_rht, uint32_t* __restrict__ flags) {
+    __shared__ __align__(16) uint32_t tile[kGaRows][kGaWords];
     __shared__ uint32_t red[8];
-    const int64_t cpr = cols >> 1;
-    const int64_t groups = rows >> 4;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int tid = threadIdx.x;
+    const int64_t ntr = (rows + kGaRows - 1) / kGaRows, ntc = (cols + 2 * kGaWords - 1) / (2 * kGaWords);
+    const int64_t ntiles = ntr * ntc;
     uint32_t m = 0;
     float mr = 0.0f;
-    for (GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr); w.r < groups; w.next()) {
-        const int64_t base = (w.r << 4) * cols + (w.k << 1);
-        uint32_t x[16], d[16];
+    for (int64_t it = blockIdx.x; it < ntiles; it += gridDim.x) {
+        const int64_t r0 = (it / ntc) * kGaRows, c0 = (it % ntc) * (2 * kGaWords);
+        // 1. GeLU of the tile: chunk j = 8 bf16 at row j / 32, columns 8 (j % 32) ..
+        uint4 v[4], d[4];
+        bool ok[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            x[i] = *reinterpret_cast<const uint32_t*>(h + base + i * cols);
-            if (BWD) d[i] = *reinterpret_cast<const uint32_t*>(dg + base + i * cols);
+        for (int u = 0; u < 4; ++u) {
+            const int j = tid + 256 * u, r = j >> 5, q = j & 31;
+            ok[u] = r0 + r < rows && c0 + 8 * q < cols;
+            const int64_t off = (r0 + r) * cols + c0 + 8 * q;
+            v[u] = ok[u] ? *reinterpret_cast<const uint4*>(h + off) : make_uint4(0, 0, 0, 0);
+            if (BWD) d[u] = ok[u] ? *reinterpret_cast<const uint4*>(dg + off) : make_uint4(0, 0, 0, 0);
         }
-        uint64_t f[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t o = BWD ? f32x2_to_bf16x2(gelu_bwd_f(bf16_lo(x[i]), bf16_lo(d[i])),
-                                                     gelu_bwd_f(bf16_hi(x[i]), bf16_hi(d[i])))
-                                   : f32x2_to_bf16x2(gelu_f(bf16_lo(x[i])), gelu_f(bf16_hi(x[i])));
-            *reinterpret_cast<uint32_t*>(out + base + i * cols) = o;
-            m = __vmaxu2(m, o & 0x7FFF7FFFu);
-            f[i] = bf16x2_to_f2(o ^ sm.m[i]);
-        }
-        rht16_pairs(f);
+        for (int u = 0; u < 4; ++u) {
+            const int j = tid + 256 * u, r = j >> 5, q = j & 31;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t o[4];
+            if (BWD) {
+                const uint32_t e[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+                if (quad_in_range(v[u])) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            float a0, a1, b0, b1;
-            f2_split(f[i], a0, a1);
-            f2_split(f[i + 1], b0, b1);
-            mr = max3_abs(max3_abs(mr, a0, a1), b0, b1);
+                    for (int k = 0; k < 4; ++k) o[k] = gelu_bwd_pair(w[k], e[k]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = gelu_bwd_word(w[k], e[k]);
+                }
+            } else {
+                if (quad_in_range(v[u])) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = gelu_pair(w[k]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = gelu_word(w[k]);
+                }
+            }
+            const uint4 ov = ok[u] ? make_uint4(o[0], o[1], o[2], o[3]) : make_uint4(0, 0, 0, 0);
+            if (ok[u]) *reinterpret_cast<uint4*>(out + (r0 + r) * cols + c0 + 8 * q) = ov;
+            *reinterpret_cast<uint4*>(&tile[r][4 * q]) = ov;
+            m = __vmaxu2(m, __vmaxu2(__vmaxu2(ov.x & 0x7FFF7FFFu, ov.y & 0x7FFF7FFFu),
+                                     __vmaxu2(ov.z & 0x7FFF7FFFu, ov.w & 0x7FFF7FFFu)));
         }
+        __syncthreads();
+        // 2. the RHT amax of column pair c of 16-row group g
+        {
+            const int g = tid >> 7, c = tid & (kGaWords - 1);
+            if (r0 + 16 * g < rows && c0 + 2 * c < cols) {
+                uint64_t f[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) f[i] = bf16x2_to_f2(tile[16 * g + i][c] ^ sm.m[i]);
+                rht16_pairs(f);
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    float a0, a1, b0, b1;
+                    f2_split(f[i], a0, a1);
+                    f2_split(f[i + 1], b0, b1);
+                    mr = max3_abs(max3_abs(mr, a0, a1), b0, b1);
+                }
+            }
+        }
+        __syncthreads();   // the tile copy is free for the next tile
     }
     const uint32_t mag = max(m & 0xFFFFu, m >> 16);
     if (mag >= 0x7F80u || !(mr < __int_as_float(0x7F800000))) atomicOr(flags, kFlagNonFinite);
@@ -225,7 +358,7 @@ static int elementwise_grid(int64_t n8) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t want = (n8 + 255) / 256;
-    int64_t cap = (int64_t)sms * 8;
+    int64_t cap = (int64_t)sms * 16;
     if (want < 1) want = 1;
     return (int)(want < cap ? want : cap);
 }
@@ -252,13 +385,13 @@ cudaError_t launch_gelu_bwd(const uint16_t* h, const uint16_t* dg, uint16_t* dh,
 cudaError_t launch_gelu_amax(bool bwd, const uint16_t* h, const uint16_t* dg, uint16_t* out, int64_t rows,
                              int64_t cols, uint32_t signs, uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags,
                              cudaStream_t s) {
-    const int64_t units = (rows >> 4) * (cols >> 1);
-    if (units == 0) return cudaSuccess;
+    const int64_t tiles = ((rows + kGaRows - 1) / kGaRows) * ((cols + 2 * kGaWords - 1) / (2 * kGaWords));
+    if (rows == 0 || cols == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t want = (units + 255) / 256, cap = (int64_t)sms * 4;   // resident CTAs at <= 64 registers
-    const int grid = (int)(want < cap ? want : cap);
+    const int64_t cap = (int64_t)sms * 8;   // resident CTAs: 16.5 KiB of shared memory each
+    const int grid = (int)(tiles < cap ? tiles : cap);
     if (bwd)
         gelu_amax_kernel<true><<<grid, 256, 0, s>>>(h, dg, out, rows, cols, sign_masks(signs), amax_plain, amax_rht, flags);
     else
