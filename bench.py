@@ -44,8 +44,8 @@ FP4_FLOP_PER_CLK = 2 * 16384 * 148
 # of one ncu capture of the SM-pair GEMM at this layer's shapes, valid for the GEMM source it was
 # taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
 GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
-GEMM_TRAFFIC = {"sha256": "e3b2bc5b716eab8373581443e49d61f2ef5f5d7a5e701936d68588cc80b3f2e1",
-                "bytes_per_launch": 484.9e6}
+GEMM_TRAFFIC = {"sha256": "57d41c7d828d87d1c35f62c9df52ab77480acf4aef8e8d9e7022243001dd78fb",
+                "bytes_per_launch": 479.9e6}
 
 
 def gemm_traffic():
@@ -388,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
         "ffn_step": ffn,
         "mxfp4_step": variants["mxfp4_step"] if variants else None,
         "bf16_step": variants["bf16_step"] if variants else None,
+        "wgrad_reduce_scatter": variants["wgrad_reduce_scatter"] if variants else None,
         "gpu_launches": launches_per_step * args.steps,
         "impl": "ours",
     }
