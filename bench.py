@@ -248,6 +248,25 @@ def run_ours(args, rank, world, local_rank):
     seg = [[cev[k][i].elapsed_time(cev[k][i + 1]) for i in range(6)] for k in range(args.steps)]
     calls_ms_per_step = statistics.mean(sum(s_) for s_ in seg)
 
+    # the step with the weight's forms cached (quantized once, as between optimizer steps with
+    # gradient accumulation): nvfp4_linear_fwd skips the weight's quantize
+    cached_w = None
+    if dp is None:
+        ctx.w_cached = True
+        cev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)
+            cev2[k][0].record()
+            step(k)
+            cev2[k][1].record()
+        torch.cuda.synchronize()
+        ctx.w_cached = False
+        if nv.nvfp4_poll(ctx.ws) != 0:
+            raise RuntimeError("device status during the cached-weight steps")
+        cms = statistics.mean(a.elapsed_time(b) for a, b in cev2)
+        cached_w = {"value": job_tflops(world, cms), "unit": "TFLOPS", "ms_per_step": cms,
+                    "workload": "the same layer step with the weight's 16x16 forms cached (no weight quantize)"}
+
     gemm_ms = [s_[i] for s_ in seg for i in (2, 4, 5)]
     q_ms = sum(s_[0] + s_[1] + s_[3] for s_ in seg)
     q_bytes = args.steps * Q_BYTES_PER_ELEM * (D_OUT * D_IN + T_TOK * D_IN + T_TOK * D_OUT)
@@ -371,6 +390,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_instruction_rate_at_clock": achieved / inst_peak if inst_peak else None,
                      "per_launch_flop": FLOP_GEMM, "avg_launch_ms": gemm_avg_ms},
         "quantize": {"gbs": q_gbs, "unit": "GB/s", "peak_hbm_gbs": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
+                     "frac_of_8000_gbs": q_gbs / 8000.0,
+                     "bound": {"X": "instruction issue", "W": "instruction issue",
+                               "dY": "integer (ALU) pipe: Philox draws and the exact SR encode"},
                      "bytes_per_elem": Q_BYTES_PER_ELEM, "peak_basis": peak_kind,
                      "per_call_ms": {"X": statistics.mean(s_[0] for s_ in seg), "W": statistics.mean(s_[1] for s_ in seg),
                                      "dY": statistics.mean(s_[3] for s_ in seg)},
@@ -382,6 +404,7 @@ def run_ours(args, rank, world, local_rank):
                         "dgrad": FLOP_GEMM / statistics.mean(s_[4] for s_ in seg) / 1e9,
                         "wgrad": FLOP_GEMM / statistics.mean(s_[5] for s_ in seg) / 1e9},
         "calls_ms_per_step": calls_ms_per_step,
+        "cached_w_step": cached_w,
         "clocks": clocks,
         "e2e": e2e,
         "c1_small_fprop": c1_latency(nv, dev) if args.c1 else None,
