@@ -49,12 +49,6 @@ __device__ __forceinline__ float normal_cdf(float h) {
 
 __device__ __forceinline__ float gelu_f(float h) { return h * normal_cdf(h); }
 
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2c(float v) { return f2(v, v); }
 __device__ __forceinline__ float rcp_approx(float x) {
     float r;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));

@@ -55,6 +55,12 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2c(float v) { return f2(v, v); }
 // the bf16 pair of a 32-bit word (low half = first element) widened to an fp32 pair (exact)
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
     return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
@@ -95,46 +101,45 @@ __device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */)
     return (uint32_t)ceilf(__fmul_rn(__uint_as_float(a), 131072.0f));
 }
 
-// The same decision without computing the threshold, on a = min(|u|, 6) (6 itself encodes 7):
-//   a in [1, 6]:  r16 < (m & 0x3FFFFF) / 2^6  <=>  (m & 0x3FFFFF) + (0x3FFFFF - 64 r16) carries into
-//                 bit 22, so the code is ((bits(a) + 0x3FFFFF - 64 r16) >> 22) - 252 (the code of
-//                 the lower neighbour is (bits(a) >> 22) - 252);
-//   a in [0, 1):  with c = ceil(a * 2^17) (exact: a * 2^17 is one exact product, and adding 2^23
-//                 rounding upward lands on 2^23 + c), the grid is {0, .5, 1} in steps of 2^16 units
-//                 of c, and the code is (c + 65535 - r16) >> 16: below .5 that is 1 iff r16 < c,
-//                 from .5 up it is 1 + [r16 < c - 65536].
-__device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
-    const uint32_t b = __float_as_uint(u);
-    const float af = fminf(fabsf(u), 6.0f);
-    const uint32_t a = __float_as_uint(af);
-    const uint32_t hi = (a + (0x3FFFFFu - (252u << 22)) - (r16 << 6)) >> 22;
-    const uint32_t cb = __float_as_uint(__fadd_ru(__fmul_rn(af, 131072.0f), 8388608.0f));   // 0x4B000000 + c
-    const uint32_t lo = (cb + (65535u - 0x4B000000u) - r16) >> 16;
-    const uint32_t code = a >= 0x3F800000u ? hi : lo;
-    return ((b >> 28) & 8u) | code;
+// The same decision without computing the threshold, as exact fp32 arithmetic on a pair (two
+// elements per f32x2 instruction, on the multiply-add pipe).  With s the grid step of |u|'s cell
+// (1/2 below 2, 1 on [2, 4), 2 from 4 up), |u| goes up iff r16 < ceil(f 2^16) with f = (|u| - lo)/s,
+// i.e. iff f 2^16 > r16, i.e. iff w = |u| - s r16 / 2^16 > lo; and since w lies in (lo - s, |u|],
+// the rounded value is s * ceil(w / s):
+//   - s = 2^max(e, 0) / 2 for |u| in [2^e, 2^(e+1)), read from the exponent bits;
+//   - w is one fused multiply-add.  It is exact from |u| = 1/2 up (|u| and s r16 / 2^16 are both
+//     multiples of |u|'s ulp, and so is w, within |u|'s binade or the one below); below 1/2 it
+//     may round but keeps its sign and zero, which is all the step-1/2 ceiling there reads;
+//   - the ceiling is one round-up add of 1.5 s 2^23 (whose binade has ulp s), and the subtraction
+//     of 1.5 s 2^23 that follows is exact.
+// The result is a signed grid value (the sign of u, also for a zero result), 8 where |u| > 6
+// rounded up: the hardware RNE conversion to E2M1 then encodes it exactly (8 saturates to 6).
+// rb_lo / rb_hi are the fp32 bits of 2^23 + r16 (sr_field_bits).
+__device__ __forceinline__ uint32_t sr_field_bits(uint32_t word, bool high) {
+    // 2^23 + the low (high = false) or the high 16-bit field of a Philox word, as fp32 bits
+    return __byte_perm(word, 0x4B000000u, high ? 0x7432u : 0x7410u);
 }
-
-// The same decision for a pair of values (lo, hi) with their own 16-bit random fields; the
-// round-up add of the |u| < 1 branch is one f32x2 instruction.  Returns lo's code in bits [0,4)
-// and hi's in bits [4,8).
-__device__ __forceinline__ uint32_t e2m1_sr_pair(uint64_t u, uint32_t r_lo, uint32_t r_hi) {
+__device__ __forceinline__ uint64_t e2m1_sr_values(uint64_t u, uint32_t rb_lo, uint32_t rb_hi) {
     float ul, uh;
     f2_split(u, ul, uh);
-    const float afl = fminf(fabsf(ul), 6.0f), afh = fminf(fabsf(uh), 6.0f);
-    uint64_t cb2;
-    asm("fma.rp.f32x2 %0, %1, %2, %3;"
-        : "=l"(cb2)
-        : "l"(f2(afl, afh)), "l"(f2(131072.0f, 131072.0f)), "l"(f2(8388608.0f, 8388608.0f)));
-    float cbl, cbh;
-    f2_split(cb2, cbl, cbh);
-    const uint32_t al = __float_as_uint(afl), ah = __float_as_uint(afh);
-    const uint32_t hil = (al + (0x3FFFFFu - (252u << 22)) - (r_lo << 6)) >> 22;
-    const uint32_t hih = (ah + (0x3FFFFFu - (252u << 22)) - (r_hi << 6)) >> 22;
-    const uint32_t lol = (__float_as_uint(cbl) + (65535u - 0x4B000000u) - r_lo) >> 16;
-    const uint32_t loh = (__float_as_uint(cbh) + (65535u - 0x4B000000u) - r_hi) >> 16;
-    const uint32_t cl = (al >= 0x3F800000u ? hil : lol) | ((__float_as_uint(ul) >> 28) & 8u);
-    const uint32_t ch = (ah >= 0x3F800000u ? hih : loh) | ((__float_as_uint(uh) >> 28) & 8u);
-    return cl | (ch << 4);
+    const float el = fmaxf(__uint_as_float(__float_as_uint(ul) & 0x7F800000u), 1.0f);   // 2^max(e, 0)
+    const float eh = fmaxf(__uint_as_float(__float_as_uint(uh) & 0x7F800000u), 1.0f);
+    const uint64_t nsq = f2_mul(f2(el, eh), f2c(-0x1p-17f));                              // -s / 2^16
+    const uint64_t r = f2_sub(f2(__uint_as_float(rb_lo), __uint_as_float(rb_hi)), f2c(8388608.0f));   // r16
+    const uint64_t w = f2_fma(nsq, r, f2(fabsf(ul), fabsf(uh)));
+    const uint64_t m = f2_mul(nsq, f2c(-0x1.8p+39f));                                     // 1.5 s 2^23
+    uint64_t t;
+    asm("add.rp.f32x2 %0, %1, %2;" : "=l"(t) : "l"(w), "l"(m));
+    float vl, vh;
+    f2_split(f2_sub(t, m), vl, vh);
+    return f2(copysignf(vl, ul), copysignf(vh, uh));
+}
+// One element: its code in bits [0, 4)
+__device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
+    const uint32_t rb = 0x4B000000u | (r16 & 0xFFFFu);
+    float vl, vh;
+    f2_split(e2m1_sr_values(f2(u, u), rb, rb), vl, vh);
+    return e2m1x2_rne(vl, vh) & 15u;
 }
 
 // ---------------------------------------------------------------------------------------

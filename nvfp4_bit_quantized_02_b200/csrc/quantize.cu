@@ -173,17 +173,20 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
 // A persistent CTA of 256 threads walks 64-row x 256-column tiles (in reverse order of the
 // amax pass).  Each tile is brought into shared memory by one 2D TMA copy (double-buffered:
 // the next tile's copy is in flight while this one is processed) and then consumed in phases
-// whose thread mappings each suit one job, so no thread holds more than one 16-element group:
+// whose thread mappings each suit one job:
 //   T  (16x16) the tile scales: 4 threads per 16x16 tile, two shuffles;
-//   R  (ROW form) one thread per 16-byte chunk (row, 8 columns); a 1x16 block is a lane pair
-//      (one shuffle); the Philox call of the chunk (stream_row) is made in place; each lane
-//      stores 4 code bytes (a warp writes 128 contiguous bytes) and every 4 blocks' scales
-//      leave as one 32-bit store;
-//   C  (COL form) one thread per (column, 16-row group): 16 values read down a column of the
-//      tile, optional 16-point RHT, block scale, codes staged in shared memory.  The SR fields
-//      of a form element are indexed by its position in the form, so the 16 elements of a
-//      COL block are two whole Philox calls made in place;
+//   R  (ROW form) one thread per 1x16 block: two 16-byte shared loads, the block scale, the 8
+//      element pairs scaled as f32x2, 8 code bytes per store; lanes 4a..4a+3 hold four
+//      consecutive blocks of a row, whose scales leave as one 32-bit store;
+//   C  (COL form) one thread per (column pair, 16-row group): 16 four-byte shared loads give
+//      both columns down the group, which stay paired through the optional 16-point RHT, the
+//      block amax and the scaling; codes are staged in shared memory;
 //   S  (COL form) the staged codes and scales leave as 16-byte (or 8-byte) row segments.
+// The rounding mode is a template parameter (one mode per call).  Under SR the Philox fields of
+// a block are drawn in place (the fields of a form element are indexed by its position in the
+// form, so a COL block's 16 elements are two whole Philox calls), the values are rounded onto the
+// E2M1 grid as exact fp32 numbers (e2m1_sr_values), and both modes then encode with the same
+// hardware RNE conversion.
 // Per-CTA tables hold r_b = S_enc / dec(c) for the 127 finite E4M3 codes (one IEEE division
 // each, identical to dividing per block).
 // ---------------------------------------------------------------------------------------
@@ -275,7 +278,7 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
     return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
-template <bool ROW, bool COL>
+template <bool ROW, bool COL, bool SR>
 __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                      const __grid_constant__ QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -293,7 +296,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
     const int64_t ntr = (rows + kTileRows - 1) / kTileRows;
     const int64_t ntc = (cols + kTileCols - 1) / kTileCols;
     const int64_t ntiles = ntr * ntc;
-    const bool sr_row = ROW && p.sr_row, sr_col = COL && p.sr_col, rht = COL && p.rht_col, b16 = p.block16 != 0;
+    constexpr bool sr_row = ROW && SR, sr_col = COL && SR;
+    const bool rht = COL && p.rht_col, b16 = p.block16 != 0;
 
     const float senc_r = encode_scale(__uint_as_float(ROW ? *p.amax_row : 0u));
     const float senc_c = encode_scale(__uint_as_float(COL ? *p.amax_col : 0u));
@@ -405,6 +409,9 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                 }
                 const uint64_t mm = f2(mult, mult);
                 uint32_t byte[8];
+                uint64_t uv[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) uv[q] = f2_mul(bf16x2_to_f2(w[q]), mm);
                 if (sr_row) {
                     const uint64_t g0 = ((uint64_t)(p.row_offset + gr) * (uint64_t)cols + (uint64_t)gc) >> 3;
                     const U4 ra = sr_words_p(p, p.stream_row, g0);
@@ -412,14 +419,13 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     const uint32_t rr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        byte[q] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[q]), mm), rr[q] & 0xFFFFu, rr[q] >> 16);
-                } else {
+                        uv[q] = e2m1_sr_values(uv[q], sr_field_bits(rr[q], false), sr_field_bits(rr[q], true));
+                }
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float lo, hi;
-                        f2_split(f2_mul(bf16x2_to_f2(w[q]), mm), lo, hi);
-                        byte[q] = e2m1x2_rne(lo, hi);
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    float lo, hi;
+                    f2_split(uv[q], lo, hi);
+                    byte[q] = e2m1x2_rne(lo, hi);
                 }
                 uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
                 sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
@@ -487,30 +493,17 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     const uint64_t g0 = ((uint64_t)(c_base + c) * (uint64_t)p.rows_total +
                                          (uint64_t)(p.row_offset + r_base + g * 16)) >> 3;
                     const uint64_t g1 = g0 + ((uint64_t)p.rows_total >> 3);   // column c + 1
-                    uint32_t nib[16];   // per row i: column c's code in bits [0,4), column c + 1's in [4,8)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {   // rows 8h .. 8h + 7: one Philox call per column
                         const U4 a = sr_words_p(p, p.stream_col, g0 + h), b = sr_words_p(p, p.stream_col, g1 + h);
                         const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint32_t r0 = (i & 1) ? (ra[i >> 1] >> 16) : (ra[i >> 1] & 0xFFFFu);
-                            const uint32_t r1 = (i & 1) ? (rb[i >> 1] >> 16) : (rb[i >> 1] & 0xFFFFu);
-                            nib[8 * h + i] = e2m1_sr_pair(v[8 * h + i], r0, r1);
-                        }
+                        for (int i = 0; i < 8; ++i)
+                            v[8 * h + i] = e2m1_sr_values(v[8 * h + i], sr_field_bits(ra[i >> 1], i & 1),
+                                                          sr_field_bits(rb[i >> 1], i & 1));
                     }
-                    // rows 2q, 2q + 1 -> byte q of each column's codes
-                    uint32_t bc0[8], bc1[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        bc0[q] = (nib[2 * q] & 15u) | ((nib[2 * q + 1] & 15u) << 4);
-                        bc1[q] = (nib[2 * q] >> 4) | (nib[2 * q + 1] & 0xF0u);
-                    }
-                    out[0] = pack4(bc0[0], bc0[1], bc0[2], bc0[3]);
-                    out[1] = pack4(bc0[4], bc0[5], bc0[6], bc0[7]);
-                    out[2] = pack4(bc1[0], bc1[1], bc1[2], bc1[3]);
-                    out[3] = pack4(bc1[4], bc1[5], bc1[6], bc1[7]);
-                } else {
+                }
+                {
                     uint32_t bc0[8], bc1[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -679,8 +672,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                         const U4 rw = mx_words(p, g0 + c);
                         const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            byte[4 * c + q] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), rr[q] & 0xFFFFu, rr[q] >> 16);
+                        for (int q = 0; q < 4; ++q) {
+                            float lo, hi;
+                            f2_split(e2m1_sr_values(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), sr_field_bits(rr[q], false),
+                                                    sr_field_bits(rr[q], true)),
+                                     lo, hi);
+                            byte[4 * c + q] = e2m1x2_rne(lo, hi);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -727,18 +725,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                     for (int h = 0; h < 4; ++h) {   // rows 8h .. 8h + 7: one Philox call per column
                         const U4 a = mx_words(p, g0 + h), bw = mx_words(p, g1 + h);
                         const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {bw.x, bw.y, bw.z, bw.w};
-                        uint32_t nib[8];
+                        uint64_t sv[8];   // row i: the SR values of columns c and c + 1
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint32_t r0 = (i & 1) ? (ra[i >> 1] >> 16) : (ra[i >> 1] & 0xFFFFu);
-                            const uint32_t r1 = (i & 1) ? (rb[i >> 1] >> 16) : (rb[i >> 1] & 0xFFFFu);
-                            nib[i] = e2m1_sr_pair(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), r0, r1);
-                        }
+                        for (int i = 0; i < 8; ++i)
+                            sv[i] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), sr_field_bits(ra[i >> 1], i & 1),
+                                                   sr_field_bits(rb[i >> 1], i & 1));
                         uint32_t b0[4], b1[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            b0[q] = (nib[2 * q] & 15u) | ((nib[2 * q + 1] & 15u) << 4);
-                            b1[q] = (nib[2 * q] >> 4) | (nib[2 * q + 1] & 0xF0u);
+                            float a0, a1, c0v, c1v;
+                            f2_split(sv[2 * q], a0, a1);
+                            f2_split(sv[2 * q + 1], c0v, c1v);
+                            b0[q] = e2m1x2_rne(a0, c0v);
+                            b1[q] = e2m1x2_rne(a1, c1v);
                         }
                         out[h] = pack4(b0[0], b0[1], b0[2], b0[3]);
                         out[4 + h] = pack4(b1[0], b1[1], b1[2], b1[3]);
@@ -893,8 +892,12 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
         k1 += 0xBB67AE85u;
     }
     const int smem = QuantSmem::bytes;
+    const bool sr = (row && p.sr_row) || (col && p.sr_col);   // one rounding mode per call
     void (*kern)(const CUtensorMap, const QuantParams) =
-        row && col ? quantize_tile_kernel<true, true> : row ? quantize_tile_kernel<true, false> : quantize_tile_kernel<false, true>;
+        sr ? (row && col ? quantize_tile_kernel<true, true, true> : row ? quantize_tile_kernel<true, false, true>
+                                                                       : quantize_tile_kernel<false, true, true>)
+           : (row && col ? quantize_tile_kernel<true, true, false> : row ? quantize_tile_kernel<true, false, false>
+                                                                        : quantize_tile_kernel<false, true, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
