@@ -621,20 +621,32 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
 def wgrad_reduce_scatter_fields(args, dev, flush, x, dy, dw) -> dict:
     """The wgrad GEMM (M = 20480, N = 5120, K = 8192 tokens) with its output stored (fp32), added
     into 8 row shards of 2560 rows (the epilogue of the data-parallel reduce-scatter, here into
-    local buffers) and added into one fp32 buffer (gradient accumulation); each call timed alone
-    with L2 flushed before it."""
+    local buffers) and added into one fp32 buffer (gradient accumulation); the three calls
+    interleaved, each timed alone with L2 flushed before it."""
     import nvfp4_bit_quantized_02_b200 as nv
     ws = nv.Workspace(dev)
     _, xc = nv.nvfp4_quantize_dual(x, mode=nv.RNE, rht_seed=3, ws=ws)
     _, dyc = nv.nvfp4_quantize_dual(dy, mode=nv.SR, rht_seed=3, sr_seed=4, stream_row=1, stream_col=2, ws=ws)
     share = D_OUT // 8
     shards = [dw[o * share:(o + 1) * share] for o in range(8)]
-    res = {}
-    for name, fn in (("stored", lambda k: nv.nvfp4_gemm(dyc, xc, out=dw, ws=ws)),
-                     ("8 owners", lambda k: nv.nvfp4_gemm_reduce_scatter(dyc, xc, shards, share, ws=ws)),
-                     ("1 owner", lambda k: nv.nvfp4_gemm_reduce_scatter(dyc, xc, [dw], D_OUT, ws=ws))):
-        per, _ = time_calls([(name, fn)], args.steps, args.warmup, flush)
-        res[name] = per[name]
+    calls = (("stored", lambda: nv.nvfp4_gemm(dyc, xc, out=dw, ws=ws)),
+             ("8 owners", lambda: nv.nvfp4_gemm_reduce_scatter(dyc, xc, shards, share, ws=ws)),
+             ("1 owner", lambda: nv.nvfp4_gemm_reduce_scatter(dyc, xc, [dw], D_OUT, ws=ws)))
+    for _ in range(args.warmup):
+        for _, fn in calls:
+            fn()
+    # the three interleaved, each with L2 flushed before it, so drifts of clock or power hit all alike
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(args.steps)]
+    for k in range(args.steps):
+        for i, (_, fn) in enumerate(calls):
+            flush.fill_((k + i) & 0xFF)
+            ev[k][i][0].record()
+            fn()
+            ev[k][i][1].record()
+    torch.cuda.synchronize()
+    res = {name: statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps))
+           for i, (name, _) in enumerate(calls)}
     if nv.nvfp4_poll(ws) != 0:
         raise RuntimeError("device status in the wgrad reduce-scatter timing")
     return {"ms": res, "tflops": {k: FLOP_GEMM / v / 1e9 for k, v in res.items()},
