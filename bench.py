@@ -412,6 +412,7 @@ def run_ours(args, rank, world, local_rank):
         "mxfp4_step": variants["mxfp4_step"] if variants else None,
         "bf16_step": variants["bf16_step"] if variants else None,
         "wgrad_reduce_scatter": variants["wgrad_reduce_scatter"] if variants else None,
+        "fprop_amax_epilogue": variants["fprop_amax_epilogue"] if variants else None,
         "gpu_launches": launches_per_step * args.steps,
         "impl": "ours",
     }
@@ -615,7 +616,40 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
     del lay
     torch.cuda.empty_cache()
     out["wgrad_reduce_scatter"] = wgrad_reduce_scatter_fields(args, dev, flush, x, dy, dw)
+    out["fprop_amax_epilogue"] = fprop_amax_fields(args, dev, flush, x, w, y)
     return out
+
+
+def fprop_amax_fields(args, dev, flush, x, w, y) -> dict:
+    """The layer's fprop (Y 8192 x 20480 bf16) with Y's amax for the next quantize: the plain GEMM
+    followed by the amax pass over Y, against the GEMM whose epilogue produces the same amax words;
+    the calls interleaved, each timed with L2 flushed before it."""
+    import nvfp4_bit_quantized_02_b200 as nv
+    ws, ws_a, ws_b = nv.Workspace(dev), nv.Workspace(dev), nv.Workspace(dev)
+    xq = nv.nvfp4_quantize(x, ws=ws)
+    wq = nv.nvfp4_quantize(w, block=nv.BLOCK_16x16, ws=ws)
+    calls = (("gemm", lambda: nv.nvfp4_gemm(xq, wq, out=y, ws=ws)),
+             ("amax pass", lambda: nv.nvfp4_amax(y, True, 0, ws_a)),
+             ("gemm with amax epilogue", lambda: nv.nvfp4_gemm_amax(xq, wq, ws_b, rht_seed=0, out=y, ws=ws)))
+    for _ in range(args.warmup):
+        for _, fn in calls:
+            fn()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(args.steps)]
+    for k in range(args.steps):
+        for i, (_, fn) in enumerate(calls):
+            flush.fill_((k + i) & 0xFF)
+            ev[k][i][0].record()
+            fn()
+            ev[k][i][1].record()
+    torch.cuda.synchronize()
+    if nv.nvfp4_poll(ws) != 0 or not torch.equal(ws_a.amax_words(), ws_b.amax_words()):
+        raise RuntimeError("the epilogue amax differs from the amax pass")
+    res = {name: statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps))
+           for i, (name, _) in enumerate(calls)}
+    return {"ms": res, "saved_ms": res["gemm"] + res["amax pass"] - res["gemm with amax epilogue"],
+            "workload": "fprop 8192x20480x5120 producing Y's plain and RHT amax: GEMM + amax pass over Y, "
+                        "against the GEMM with the amax epilogue (equal words checked)"}
 
 
 def wgrad_reduce_scatter_fields(args, dev, flush, x, dy, dw) -> dict:

@@ -207,6 +207,21 @@ nvfp4_status nvfp4_gemm_reduce_scatter(const nvfp4_tensor* a, const nvfp4_tensor
                                        nvfp4_stream_t stream);
 
 /*
+ * nvfp4_gemm with bf16 output that also produces the output's amax for the quantize call that
+ * will read it (gist.science 2.A: the FP32 tensor scale comes from the amax of the whole tensor,
+ * a pass over it that the producer can take over): the plain amax of the stored bf16 D and the
+ * amax of its 16-point RHT along the rows (signs from rht_seed, the transform of the wgrad form
+ * of D as a token-major operand) are written into amax_ws's amax words, exactly as nvfp4_amax(D,
+ * rht = 1, rht_seed) would: the same fp32 operations on the same bf16 values.  A linear context
+ * whose workspace is amax_ws can then quantize D with amax_ready set, and
+ * nvfp4_quantize_dual_shard(D, 0, rows, ...) with amax_ws uses the words as they are.  amax_ws's
+ * words are reset first; a non-finite output raises the non-finite flag in ws.  Shape rules: those
+ * of nvfp4_gemm, and M % 16 == 0.
+ */
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, int64_t ldd,
+                             uint64_t rht_seed, void* amax_ws, void* ws, nvfp4_stream_t stream);
+
+/*
  * Linear layer y = x w^T with NVFP4 GEMMs (gist.science 2.B): all buffers caller-owned.
  *   xq      [T][d]   1x16 RNE           (fprop A)
  *   xq_rht  [d][T]   RHT 1x16 RNE       (wgrad B)

@@ -82,6 +82,7 @@ def _lib():
             "nvfp4_transpose_2d": ([T, T, vp], i32),
             "nvfp4_gemm": ([T, T, vp, i64, i32, vp, vp], i32),
             "nvfp4_gemm_reduce_scatter": ([T, T, c.POINTER(vp), i32, i64, i64, vp, vp], i32),
+            "nvfp4_gemm_amax": ([T, T, vp, i64, u64, vp, vp, vp], i32),
             "nvfp4_linear_fwd": ([vp, vp, vp, c.POINTER(CLinearCtx), vp], i32),
             "nvfp4_linear_bwd": ([vp, u64, vp, vp, c.POINTER(CLinearCtx), vp], i32),
             "nvfp4_gelu_fwd": ([vp, vp, i64, vp], i32),
@@ -321,6 +322,23 @@ def nvfp4_gemm(a: NVFP4Tensor, b: NVFP4Tensor, out_dtype=torch.bfloat16, out: to
     ca, cb = a.c(), b.c()
     st = _lib().nvfp4_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), out.stride(0), code, ws.ptr, _stream(stream))
     _check(st, "nvfp4_gemm")
+    return out
+
+
+def nvfp4_gemm_amax(a: NVFP4Tensor, b: NVFP4Tensor, amax_ws: Workspace, rht_seed: int = 0,
+                    out: torch.Tensor | None = None, ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """D = s_tA s_tB * A . B^T in bf16, with D's plain and RHT amax written into amax_ws (as
+    nvfp4_amax(D, True, rht_seed, amax_ws) would), ready for the quantize call that reads D."""
+    M, N = a.rows, b.rows
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.codes.device)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("nvfp4_gemm_amax writes bf16")
+    ws = ws or default_workspace()
+    ca, cb = a.c(), b.c()
+    st = _lib().nvfp4_gemm_amax(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), out.stride(0), rht_seed, amax_ws.ptr,
+                                ws.ptr, _stream(stream))
+    _check(st, "nvfp4_gemm_amax")
     return out
 
 

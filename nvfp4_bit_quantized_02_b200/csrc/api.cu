@@ -417,6 +417,26 @@ nvfp4_status nvfp4_gemm_reduce_scatter(const nvfp4_tensor* a, const nvfp4_tensor
                                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_gemm_amax(const nvfp4_tensor* a, const nvfp4_tensor* b, void* d, int64_t ldd, uint64_t rht_seed,
+                             void* amax_ws, void* ws, nvfp4_stream_t stream) {
+    if (!a || !b || !d) return NVFP4_ERR_NULL;
+    if (nvfp4_status st = check_form_buffers(a, false)) return st;
+    if (nvfp4_status st = check_form_buffers(b, false)) return st;
+    if (!ws || !amax_ws) return NVFP4_ERR_WORKSPACE;
+    const int64_t M = a->rows, N = b->rows, K = a->k;
+    if (b->k != K) return NVFP4_ERR_ARG;
+    if (M < 16 || M % 16 != 0 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return NVFP4_ERR_LIMIT;
+    if (ldd < N) return NVFP4_ERR_SHAPE;
+    if (!aligned16(d) || (ldd * 2) % 16 != 0) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_device()) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaError_t e = reset_amax(amax_ws, s)) return from_cuda(e);
+    return from_cuda(launch_gemm_nvf4_amax(a->codes, a->scales, a->tensor_scale, M, b->codes, b->scales, b->tensor_scale, N,
+                                           K, d, ldd, &ws_of(amax_ws)->amax_a, rht_signs_host(rht_seed),
+                                           &ws_of(ws)->flags, g_budget_ns.load(), s));
+}
+
 static nvfp4_status check_ctx(const nvfp4_linear_ctx* c) {
     if (!c) return NVFP4_ERR_NULL;
     if (c->T <= 0 || c->d <= 0 || c->n <= 0) return NVFP4_ERR_SHAPE;

@@ -43,6 +43,7 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "nvfp4_device.cuh"
 #include "nvfp4_internal.h"
 
 namespace nvfp4 {
@@ -286,6 +287,10 @@ struct GemmParams {
     // (o + 1) * owner_rows) are added into owner o's shard through its own tensor map
     int32_t n_owners;
     int32_t owner_rows;
+    // amax epilogue (null: off; bf16 output): the plain amax of the stored output and the amax of
+    // its 16-point RHT along the rows go to amax_out[0] and amax_out[1] (fp32 bits, atomic max)
+    uint32_t* amax_out;
+    uint32_t rht_mask[16];   // row i of a 16-row group: 0x80008000 where the RHT sign is -1
 };
 
 // The shards of a reduce-scatter epilogue: one fp32 output map per owner (a local buffer or
@@ -331,12 +336,66 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm,
 // false on abort.
 // With owner maps (the reduce-scatter epilogue) each box is added into the shard of the owner of
 // its rows instead of stored.
-template <int kSlots>
+// With p.amax_out (bf16 output) the warp also reads its staged box back, each lane one column pair
+// of both 16-row groups, for the plain and RHT amax of the output (rows >= M and columns >= N,
+// which hold padding, excluded): the same loads, sign flips, butterfly and maxima as the amax pass
+// of a quantize call over the stored tensor.
+__device__ __forceinline__ void box_amax(uint32_t sbase, int x, int y, const GemmParams& p, uint32_t& am_plain,
+                                         float& am_rht) {
+    const int lane = threadIdx.x & 31;
+    const int col = x + 2 * lane;
+    if (col >= p.N) return;
+    const uint32_t keep = col + 1 < p.N ? 0xFFFFFFFFu : 0x0000FFFFu;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        if (y + 16 * g >= p.M) break;
+        uint64_t f[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int rr = 16 * g + i;
+            uint32_t w;
+            asm volatile("ld.shared.u32 %0, [%1];"
+                         : "=r"(w)
+                         : "r"(sbase + (uint32_t)rr * 128u + ((((uint32_t)lane >> 2) ^ (uint32_t)(rr & 7)) << 4) +
+                               (((uint32_t)lane & 3u) << 2)));
+            w &= keep;
+            am_plain = __vmaxu2(am_plain, w & 0x7FFF7FFFu);
+            f[i] = bf16x2_to_f2(w ^ p.rht_mask[i]);
+        }
+        rht16_pairs(f);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            float a0, a1, b0, b1;
+            f2_split(f[i], a0, a1);
+            f2_split(f[i + 1], b0, b1);
+            am_rht = max3_abs(max3_abs(am_rht, a0, a1), b0, b1);
+        }
+    }
+}
+
+// The amax epilogue's per-warp maxima into the output words (and the non-finite flag)
+__device__ __forceinline__ void amax_flush(const GemmParams& p, uint32_t am_plain, float am_rht) {
+    uint32_t m = max(am_plain & 0xFFFFu, am_plain >> 16) << 16;
+    uint32_t mr = __float_as_uint(am_rht);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        mr = max(mr, __shfl_xor_sync(0xFFFFFFFFu, mr, o));   // non-negative floats order as integers
+    }
+    if ((threadIdx.x & 31) == 0) {
+        if (m) atomicMax(p.amax_out, m);
+        if (mr) atomicMax(p.amax_out + 1, mr);
+        if (m >= 0x7F800000u || mr >= 0x7F800000u) atomicOr(p.flags, kFlagNonFinite);
+    }
+}
+
+template <int kSlots, bool AMAX>
 __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtensorMap* owner_maps, uint8_t* store_area,
                                             uint64_t* boxgo_bar, const uint32_t (&r)[2][32], int ew, int local, int x0,
-                                            int y, const GemmParams& p, float alpha, volatile uint32_t* abort_flag) {
+                                            int y, const GemmParams& p, float alpha, volatile uint32_t* abort_flag,
+                                            uint32_t& am_plain, float& am_rht) {
     const int lane = threadIdx.x & 31;
-    const int nbox = p.out_fp32 ? 2 : 1;
+    const int nbox = (!AMAX && p.out_fp32) ? 2 : 1;   // the amax epilogue serves bf16 outputs only
     const int nb = kEpi1Warps * nbox;   // boxes per tile, a multiple of kSlots
     const uint32_t swz = (uint32_t)(lane & 7);
 #pragma unroll
@@ -377,6 +436,20 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtens
         }
         fence_async_smem();
         __syncwarp();
+        if (AMAX) {
+            // the store first, then the read-back of the box, then its release
+            if (lane == 0 && x < p.N && y < p.M) tma_store_2d(tmD, sbase, x, y);
+            if (lane == 0) bulk_commit();
+            box_amax(sbase, x, y, p, am_plain, am_rht);
+            __syncwarp();
+            if (lane == 0) {
+                bulk_wait_read_all();
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&boxgo_bar[(b + kSlots) % nb]))
+                             : "memory");
+            }
+            __syncwarp();
+            continue;
+        }
         if (lane == 0) {
             if (x < p.N && y < p.M) {
                 if (owner_maps) {
@@ -395,7 +468,7 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtens
     return true;
 }
 
-template <bool MX>
+template <bool MX, bool AMAX>
 __global__ void __launch_bounds__(kGemm1Threads, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmD, const __grid_constant__ OwnerMaps om, GemmParams p) {
@@ -554,6 +627,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         const float alpha = p.sta ? __fmul_rn(*p.sta, *p.stb) : 1.0f;   // MXFP4: no tensor scales
         int local = 0;
         bool ok = true;
+        uint32_t am_plain = 0;
+        float am_rht = 0.0f;
         for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
             int tm, tn;
             tile_coords(t, p, tm, tn);
@@ -567,9 +642,10 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(tempty_bar)) : "memory");
-            ok = store_boxes<kStoreSlots>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64, tm * kBM + q * 32,
-                                          p, alpha, abort_flag);
+            ok = store_boxes<kStoreSlots, AMAX>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64, tm * kBM + q * 32,
+                                          p, alpha, abort_flag, am_plain, am_rht);
         }
+        if (AMAX) amax_flush(p, am_plain, am_rht);
         if (lane == 0) bulk_wait_all();   // this lane's stores are in global memory before the CTA exits
     } else {
         // ------------------------------- scale warps (18..21) -------------------------------
@@ -775,7 +851,7 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, u
         : "memory");
 }
 
-template <int F>
+template <int F, bool AMAX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
     gemm_nvf4_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -948,6 +1024,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
         const uint32_t drained = smem_u32(rank == 0 ? tempty_bar : edrained_bar);
         int local = 0;
         bool ok = true;
+        uint32_t am_plain = 0;
+        float am_rht = 0.0f;
         for (int t = pair; ok && t < ntiles; t += npairs, ++local) {
             int tm, tn;
             tile_coords(t, p, tm, tn);
@@ -961,9 +1039,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(drained) : "memory");
-            ok = store_boxes<k2StoreSlots>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
-                                           tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag);
+            ok = store_boxes<k2StoreSlots, AMAX>(&tmD, p.n_owners ? om.m : nullptr, store_area, boxgo_bar, r, ew, local, tn * kBN + cq * 64,
+                                           tm * 256 + (int)rank * 128 + q * 32, p, alpha, abort_flag, am_plain, am_rht);
         }
+        if (AMAX) amax_flush(p, am_plain, am_rht);
         if (lane == 0) bulk_wait_all();
     }
 
@@ -1103,7 +1182,8 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
                                const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
                                void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
                                cudaStream_t stream, float* const* owner_d = nullptr, int n_owners = 0,
-                               int64_t owner_rows = 0) {
+                               int64_t owner_rows = 0, uint32_t* amax_out = nullptr, uint32_t rht_signs = 0) {
+    if (amax_out && (out_fp32 || n_owners > 0 || M % 16 != 0)) return cudaErrorInvalidValue;
     if (n_owners < 0 || n_owners > kMaxOwners || (n_owners > 0 && (!out_fp32 || owner_rows < 32 || owner_rows % 32 != 0 ||
                                                                    (M + owner_rows - 1) / owner_rows != n_owners)))
         return cudaErrorInvalidValue;
@@ -1115,7 +1195,7 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         om = &om_local;
         d = owner_d[0];   // the plain output map is built but never written
     }
-    GemmParams p;
+    GemmParams p{};   // value-initialized: every field not set below is zero (no owners, no amax)
     p.sfa = a_scales;
     p.sfb = b_scales;
     p.sta = a_st;
@@ -1138,6 +1218,8 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     p.budget_ns = budget_ns;
     p.n_owners = n_owners;
     p.owner_rows = (int32_t)owner_rows;
+    p.amax_out = amax_out;
+    for (int i = 0; i < 16; ++i) p.rht_mask[i] = ((rht_signs >> i) & 1u) ? 0x80008000u : 0u;
     const int sms = sm_count();
     // SM-pair tiles for M >= 256 (fewer operand bytes per SM per K block, a deeper ring);
     // NVFP4_GEMM_VARIANT=1sm selects the 1-SM kernel for every shape (read on every call)
@@ -1145,7 +1227,9 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     const bool force_1sm = variant && strcmp(variant, "1sm") == 0;
     if (!force_1sm && M >= 256 && sms >= 2) {
         static std::atomic<uint64_t> attr_2sm{0};
-        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4>), k2Smem, attr_2sm))
+        auto kern2 = amax_out ? gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4, true> : gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4, false>;
+        static std::atomic<uint64_t> attr_2sm_amax{0};
+        if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern2), k2Smem, amax_out ? attr_2sm_amax : attr_2sm))
             return e;
         CUtensorMap ta2, tb2;
         if (!make_code_map(&ta2, a_codes, M, K, 128) || !make_code_map(&tb2, b_codes, N, K, 128)) return cudaErrorInvalidValue;
@@ -1157,12 +1241,14 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         if (!make_out_map(&td2, d, M, N, ldd, out_fp32) || !make_sf_map(&tsa, a_scales, p.sfa_row_tiles, p.nkt, 1, sfe) ||
             !make_sf_map(&tsb, b_scales, p.sfb_row_tiles, p.nkt, 2, sfe))
             return cudaErrorInvalidValue;
-        gemm_nvf4_2sm_kernel<MX ? kMXF4 : kNVF4><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2,
-                                                                                                      *om, p);
+        kern2<<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta2, tb2, tsa, tsb, td2, *om, p);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> attr_1sm{0};
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_kernel<MX>), kGemmSmem, attr_1sm)) return e;
+    auto kern1 = amax_out ? gemm_nvf4_kernel<MX, true> : gemm_nvf4_kernel<MX, false>;
+    static std::atomic<uint64_t> attr_1sm_amax{0};
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern1), kGemmSmem, amax_out ? attr_1sm_amax : attr_1sm))
+        return e;
     CUtensorMap ta, tb;
     if (!make_code_map(&ta, a_codes, M, K, kBM) || !make_code_map(&tb, b_codes, N, K, kBN))
         return cudaErrorInvalidValue;
@@ -1170,7 +1256,7 @@ static cudaError_t launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     CUtensorMap td;
     if (!make_out_map(&td, d, M, N, ldd, out_fp32)) return cudaErrorInvalidValue;
-    gemm_nvf4_kernel<MX><<<grid, kGemm1Threads, kGemmSmem, stream>>>(ta, tb, td, *om, p);
+    kern1<<<grid, kGemm1Threads, kGemmSmem, stream>>>(ta, tb, td, *om, p);
     return cudaGetLastError();
 }
 
@@ -1188,6 +1274,14 @@ cudaError_t launch_gemm_nvf4_reduce_scatter(const uint8_t* a_codes, const uint8_
                                             uint32_t* flags, uint64_t budget_ns, cudaStream_t stream) {
     return launch_gemm<false>(a_codes, a_scales, a_st, M, b_codes, b_scales, b_st, N, K, nullptr, ldd, true, flags,
                               budget_ns, stream, shards, n_owners, owner_rows);
+}
+
+cudaError_t launch_gemm_nvf4_amax(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
+                                  const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
+                                  void* d, int64_t ldd, uint32_t* amax_out, uint32_t rht_signs, uint32_t* flags,
+                                  uint64_t budget_ns, cudaStream_t stream) {
+    return launch_gemm<false>(a_codes, a_scales, a_st, M, b_codes, b_scales, b_st, N, K, d, ldd, false, flags, budget_ns,
+                              stream, nullptr, 0, 0, amax_out, rht_signs);
 }
 
 // MXFP4 operands carry no tensor scale (null scale pointers: the epilogue's factor is 1)
@@ -1219,8 +1313,9 @@ cudaError_t launch_gemm_bf16(const uint16_t* a, int64_t lda, const uint16_t* b, 
                              int64_t K, void* d, int64_t ldd, bool out_fp32, uint32_t* flags, uint64_t budget_ns,
                              cudaStream_t stream) {
     static std::atomic<uint64_t> attr{0};
-    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_2sm_kernel<kBF16>), k2Smem, attr)) return e;
-    GemmParams p;
+    if (cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemm_nvf4_2sm_kernel<kBF16, false>), k2Smem, attr))
+        return e;
+    GemmParams p{};   // value-initialized: every field not set below is zero (no owners, no amax)
     std::memset(&p, 0, sizeof(p));
     p.d = d;
     p.ldd = ldd;
@@ -1246,7 +1341,7 @@ cudaError_t launch_gemm_bf16(const uint16_t* a, int64_t lda, const uint16_t* b, 
     const int64_t pairs = ntiles < sms / 2 ? ntiles : sms / 2;
     // the scale maps are not read by the bf16 instantiation; valid maps are passed in their place
     static const OwnerMaps no_owners{};
-    gemm_nvf4_2sm_kernel<kBF16><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta, tb, ta, tb, td, no_owners, p);
+    gemm_nvf4_2sm_kernel<kBF16, false><<<(unsigned)(2 * pairs), k2Threads, k2Smem, stream>>>(ta, tb, ta, tb, td, no_owners, p);
     return cudaGetLastError();
 }
 

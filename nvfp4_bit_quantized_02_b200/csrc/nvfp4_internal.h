@@ -98,6 +98,10 @@ cudaError_t launch_gemm_nvf4_reduce_scatter(const uint8_t* a_codes, const uint8_
                                             const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N,
                                             int64_t K, float* const* shards, int n_owners, int64_t owner_rows, int64_t ldd,
                                             uint32_t* flags, uint64_t budget_ns, cudaStream_t stream);
+cudaError_t launch_gemm_nvf4_amax(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_st, int64_t M,
+                                  const uint8_t* b_codes, const uint8_t* b_scales, const float* b_st, int64_t N, int64_t K,
+                                  void* d, int64_t ldd, uint32_t* amax_out, uint32_t rht_signs, uint32_t* flags,
+                                  uint64_t budget_ns, cudaStream_t stream);
 cudaError_t launch_gemm_mxf4(const uint8_t* a_codes, const uint8_t* a_scales, int64_t M, const uint8_t* b_codes,
                              const uint8_t* b_scales, int64_t N, int64_t K, void* d, int64_t ldd, bool out_fp32,
                              uint32_t* flags, uint64_t budget_ns, cudaStream_t stream);
