@@ -243,6 +243,15 @@ typedef struct {
      * (nvfp4_gelu_fwd_amax, nvfp4_gelu_bwd_amax, or nvfp4_amax + a reduction); the call then
      * skips its amax pass and sets the field back to 0 */
     int32_t amax_ready;
+    /* optional: the amax words of this layer's outputs for the contexts that will quantize them.
+     * Non-null y_amax_ws makes nvfp4_linear_fwd's fprop GEMM also write y's plain amax and its RHT
+     * amax (signs from y_rht_seed) into that workspace (nvfp4_gemm_amax; T % 16 == 0 holds); the
+     * consuming context (y is its x) then sets amax_ready.  dx_amax_ws / dx_rht_seed do the same
+     * for dx in nvfp4_linear_bwd (dx is the consuming context's dy).  Null: off. */
+    void* y_amax_ws;
+    uint64_t y_rht_seed;
+    void* dx_amax_ws;
+    uint64_t dx_rht_seed;
 } nvfp4_linear_ctx;
 
 /* Forward: quantize X (both forms), quantize W (16x16, both layouts) unless cached, then

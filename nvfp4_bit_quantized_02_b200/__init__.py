@@ -52,7 +52,8 @@ class CLinearCtx(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("n", ctypes.c_int64), ("rht_seed", ctypes.c_uint64),
                 ("xq", CTensor), ("xq_rht", CTensor), ("wq", CTensor), ("wqt", CTensor), ("dyq", CTensor),
                 ("dyq_rht", CTensor), ("ws", ctypes.c_void_p), ("w_cached", ctypes.c_int32),
-                ("amax_ready", ctypes.c_int32)]
+                ("amax_ready", ctypes.c_int32), ("y_amax_ws", ctypes.c_void_p), ("y_rht_seed", ctypes.c_uint64),
+                ("dx_amax_ws", ctypes.c_void_p), ("dx_rht_seed", ctypes.c_uint64)]
 
 
 _L = None
@@ -544,6 +545,16 @@ class LinearContext:
     @amax_ready.setter
     def amax_ready(self, v: bool):
         self.ctx.amax_ready = 1 if v else 0
+
+    def feed(self, consumer: "LinearContext"):
+        """This layer's y is consumer's x and consumer's dx is this layer's dy (a stack of layers):
+        this layer's fprop GEMM writes y's amax words into consumer's workspace, and consumer's
+        dgrad GEMM writes dx's into this layer's, so the consuming quantize calls skip their amax
+        passes (the caller sets amax_ready on the consuming context before its call)."""
+        self.ctx.y_amax_ws = consumer.ws.ptr
+        self.ctx.y_rht_seed = consumer.ctx.rht_seed
+        consumer.ctx.dx_amax_ws = self.ws.ptr
+        consumer.ctx.dx_rht_seed = self.ctx.rht_seed
 
 
 # ---------------------------------------------------------------------------------------

@@ -458,6 +458,8 @@ nvfp4_status nvfp4_linear_fwd(const void* x, const void* w, void* y, nvfp4_linea
         st = nvfp4_quantize_weight(w, ctx->n, ctx->d, ctx->d, &ctx->wq, &ctx->wqt, ctx->ws, stream);
         if (st) return st;
     }
+    if (ctx->y_amax_ws)
+        return nvfp4_gemm_amax(&ctx->xq, &ctx->wq, y, ctx->n, ctx->y_rht_seed, ctx->y_amax_ws, ctx->ws, stream);
     return nvfp4_gemm(&ctx->xq, &ctx->wq, y, ctx->n, NVFP4_OUT_BF16, ctx->ws, stream);
 }
 
@@ -471,7 +473,9 @@ nvfp4_status nvfp4_linear_bwd(const void* dy, uint64_t sr_seed, void* dx, float*
                                          NVFP4_STREAM_WGRAD, &ctx->dyq, &ctx->dyq_rht, ctx->ws, stream, 0, ctx->T, !ready);
     if (st) return st;
     if (dx) {
-        st = nvfp4_gemm(&ctx->dyq, &ctx->wqt, dx, ctx->d, NVFP4_OUT_BF16, ctx->ws, stream);
+        st = ctx->dx_amax_ws ? nvfp4_gemm_amax(&ctx->dyq, &ctx->wqt, dx, ctx->d, ctx->dx_rht_seed, ctx->dx_amax_ws,
+                                               ctx->ws, stream)
+                             : nvfp4_gemm(&ctx->dyq, &ctx->wqt, dx, ctx->d, NVFP4_OUT_BF16, ctx->ws, stream);
         if (st) return st;
     }
     if (dw) {

@@ -79,6 +79,12 @@ def test_validation_before_any_device_work(L):
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), None, 128, 0, ws, None) == 1
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 129, 0, ws, None) == 2
     assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 100, 0, ws, None) == 3
+    # the amax epilogue: its workspace, M % 16, bf16 row alignment
+    assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 128, 0, None, ws, None) == 5
+    a.rows = 120
+    assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, ws, None) == 3
+    a.rows = 128
+    assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 132, 0, ws, ws, None) == 2
     # linear: shapes must be multiples of 64
     ctx = nv.CLinearCtx()
     ctx.T, ctx.d, ctx.n, ctx.ws = 100, 64, 64, 16

@@ -94,3 +94,34 @@ def test_epilogue_amax_argument_errors():
     with pytest.raises(m.NVFP4Error) as e:
         m.nvfp4_gemm_amax(a, b, m.Workspace())
     assert e.value.status == 3
+
+
+def test_stacked_layers_with_fed_amax_equal_the_plain_stack():
+    # two layers, the second reading the first's y: with feed() the first's fprop GEMM writes y's
+    # amax words for the second's quantize and the second's dgrad GEMM writes dx's for the first's
+    # backward, so both skip an amax pass; every output equals the stack without it, bit for bit
+    m = nv()
+    T, d, n = 256, 320, 512
+    x = to_device_bf16(synth.activations(T, d, seed=0, outlier_frac=0.01))
+    w1 = to_device_bf16(synth.weights(n, d, seed=1))
+    w2 = to_device_bf16(synth.weights(d, n, seed=3))
+    dy2 = to_device_bf16(synth.grad_output(T, d, seed=4))
+
+    def run(fed):
+        l1 = m.LinearContext(T, d, n, rht_seed=3)
+        l2 = m.LinearContext(T, n, d, rht_seed=8)
+        if fed:
+            l1.feed(l2)
+        y1 = m.nvfp4_linear_fwd(l1, x, w1)
+        l2.amax_ready = fed
+        y2 = m.nvfp4_linear_fwd(l2, y1, w2)
+        dx2, dw2 = m.nvfp4_linear_bwd(l2, dy2, 5)
+        l1.amax_ready = fed
+        dx1, dw1 = m.nvfp4_linear_bwd(l1, dx2, 6)
+        torch.cuda.synchronize()
+        assert m.nvfp4_poll(l1.ws) == 0 and m.nvfp4_poll(l2.ws) == 0
+        assert not l1.amax_ready and not l2.amax_ready
+        return [y1, y2, dx2, dw2, dx1, dw1]
+
+    for name, a, b in zip(("y1", "y2", "dx2", "dw2", "dx1", "dw1"), run(False), run(True)):
+        assert torch.equal(a, b), name
