@@ -337,13 +337,25 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& tm,
 // With owner maps (the reduce-scatter epilogue) each box is added into the shard of the owner of
 // its rows instead of stored.
 // With p.amax_out (bf16 output) the warp also reads its staged box back, each lane one column pair
-// of both 16-row groups, for the plain and RHT amax of the output (rows >= M and columns >= N,
-// which hold padding, excluded): the same loads, sign flips, butterfly and maxima as the amax pass
-// of a quantize call over the stored tensor.
-__device__ __forceinline__ void box_amax(uint32_t sbase, int x, int y, const GemmParams& p, uint32_t& am_plain,
-                                         float& am_rht) {
-    const int lane = threadIdx.x & 31;
-    const int col = x + 2 * lane;
+// of both 16-row groups (box_read: 32 shared loads, after which the slot can be released), and
+// then takes the plain and RHT amax of those words (words_amax), excluding rows >= M and columns
+// >= N, which hold padding: the same sign flips, butterfly and maxima as the amax pass of a
+// quantize call over the stored tensor.
+__device__ __forceinline__ void box_read(uint32_t sbase, uint32_t (&w)[2][16]) {
+    const uint32_t lane = threadIdx.x & 31;
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t rr = (uint32_t)(16 * g + i);
+            asm volatile("ld.shared.u32 %0, [%1];"
+                         : "=r"(w[g][i])
+                         : "r"(sbase + rr * 128u + (((lane >> 2) ^ (rr & 7u)) << 4) + ((lane & 3u) << 2)));
+        }
+}
+__device__ __forceinline__ void words_amax(const uint32_t (&w)[2][16], int x, int y, const GemmParams& p,
+                                           uint32_t& am_plain, float& am_rht) {
+    const int col = x + 2 * (threadIdx.x & 31);
     if (col >= p.N) return;
     const uint32_t keep = col + 1 < p.N ? 0xFFFFFFFFu : 0x0000FFFFu;
 #pragma unroll
@@ -352,15 +364,9 @@ __device__ __forceinline__ void box_amax(uint32_t sbase, int x, int y, const Gem
         uint64_t f[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const int rr = 16 * g + i;
-            uint32_t w;
-            asm volatile("ld.shared.u32 %0, [%1];"
-                         : "=r"(w)
-                         : "r"(sbase + (uint32_t)rr * 128u + ((((uint32_t)lane >> 2) ^ (uint32_t)(rr & 7)) << 4) +
-                               (((uint32_t)lane & 3u) << 2)));
-            w &= keep;
-            am_plain = __vmaxu2(am_plain, w & 0x7FFF7FFFu);
-            f[i] = bf16x2_to_f2(w ^ p.rht_mask[i]);
+            const uint32_t v = w[g][i] & keep;
+            am_plain = __vmaxu2(am_plain, v & 0x7FFF7FFFu);
+            f[i] = bf16x2_to_f2(v ^ p.rht_mask[i]);
         }
         rht16_pairs(f);
 #pragma unroll
@@ -437,10 +443,11 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtens
         fence_async_smem();
         __syncwarp();
         if (AMAX) {
-            // the store first, then the read-back of the box, then its release
+            // the store first, then the read-back of the box and its release, then the maxima
             if (lane == 0 && x < p.N && y < p.M) tma_store_2d(tmD, sbase, x, y);
             if (lane == 0) bulk_commit();
-            box_amax(sbase, x, y, p, am_plain, am_rht);
+            uint32_t wv[2][16];
+            box_read(sbase, wv);
             __syncwarp();
             if (lane == 0) {
                 bulk_wait_read_all();
@@ -448,6 +455,7 @@ __device__ __forceinline__ bool store_boxes(const CUtensorMap* tmD, const CUtens
                              : "memory");
             }
             __syncwarp();
+            words_amax(wv, x, y, p, am_plain, am_rht);
             continue;
         }
         if (lane == 0) {
