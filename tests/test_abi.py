@@ -85,6 +85,11 @@ def test_validation_before_any_device_work(L):
     assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, ws, None) == 3
     a.rows = 128
     assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 132, 0, ws, ws, None) == 2
+    # sizes past the fixed limit (2^30 rows or K) are refused before any device work
+    a.rows = (1 << 30) + 16
+    assert L.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, None) == 10
+    assert L.nvfp4_gemm_amax(ctypes.byref(a), ctypes.byref(b), d, 128, 0, ws, ws, None) == 10
+    a.rows = 128
     # linear: shapes must be multiples of 64
     ctx = nv.CLinearCtx()
     ctx.T, ctx.d, ctx.n, ctx.ws = 100, 64, 64, 16
