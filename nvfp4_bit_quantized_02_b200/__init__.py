@@ -555,6 +555,9 @@ class LinearContext:
         self.ctx.y_rht_seed = consumer.ctx.rht_seed
         consumer.ctx.dx_amax_ws = self.ws.ptr
         consumer.ctx.dx_rht_seed = self.ctx.rht_seed
+        # each context now holds the other's workspace address: keep both workspaces alive
+        self._feeds = consumer
+        consumer._fed_by = self
 
 
 # ---------------------------------------------------------------------------------------
