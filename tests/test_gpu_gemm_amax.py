@@ -125,3 +125,21 @@ def test_stacked_layers_with_fed_amax_equal_the_plain_stack():
 
     for name, a, b in zip(("y1", "y2", "dx2", "dw2", "dx1", "dw1"), run(False), run(True)):
         assert torch.equal(a, b), name
+
+
+def test_non_finite_output_raises_the_flag():
+    # operands near the top of bf16's range overflow the fp32 accumulation to inf: the epilogue's
+    # plain amax sees it and raises the non-finite flag in the call's workspace, as the amax pass
+    # over the stored output does in its own
+    m = nv()
+    M, N, K = 256, 256, 256
+    x = torch.full((M, K), 1e19, dtype=torch.bfloat16, device="cuda")
+    w = torch.full((N, K), 1e19, dtype=torch.bfloat16, device="cuda")
+    a, b = m.nvfp4_quantize(x, along=0), m.nvfp4_quantize(w, along=0, block=m.BLOCK_16x16)
+    ws_amax, ws, ws_ref = m.Workspace(), m.Workspace(), m.Workspace()
+    d = m.nvfp4_gemm_amax(a, b, ws_amax, ws=ws)
+    m.nvfp4_amax(d, True, 0, ws_ref)
+    torch.cuda.synchronize()
+    assert torch.isinf(d.float()).all()
+    assert m.nvfp4_poll(ws) == 7 and m.nvfp4_poll(ws_ref) == 7
+    assert int(ws_amax.amax_words()[0]) == 0x7F800000
