@@ -5,9 +5,10 @@
 // (2.B.4): round-to-nearest-even, or stochastic rounding for gradients.  Rotation (2.B.2): a
 // seeded 16-point Random Hadamard Transform.
 //
-// Every fp32 operation whose result decides a code is written as one IEEE operation in
-// round-to-nearest (explicit __fdiv_rn / __fmul_rn / __fadd_rn / __fsub_rn), so that codes
-// and scales are reproducible bit for bit.
+// Every fp32 operation whose result decides a code is written as one IEEE operation with an
+// explicit rounding mode (__fdiv_rn / __fmul_rn / __fadd_rn / __fsub_rn, the f32x2 .rn forms, and
+// the one round-up add of the stochastic rounding), never contracted or reassociated by the
+// compiler, so that codes and scales are reproducible bit for bit.
 #pragma once
 
 #include <cstdint>
