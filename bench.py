@@ -58,12 +58,22 @@ def gemm_traffic():
 
 
 def load_peaks():
+    """The measured peaks of this machine's B200s, else the earlier measurement used as fallback
+    (per key: a missing or malformed entry falls back alone, and the basis says so)."""
+    fallback = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
     try:
         with open(PEAKS_FILE) as f:
             p = json.load(f)
-        return p, "measured"
-    except OSError:
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+    except (OSError, ValueError):
+        return fallback, "fallback"
+    out, kind = {}, "measured"
+    for k, v in fallback.items():
+        x = p.get(k) if isinstance(p, dict) else None
+        if isinstance(x, (int, float)) and not isinstance(x, bool) and x > 0:
+            out[k] = float(x)
+        else:
+            out[k], kind = v, "measured (fallback for missing entries)"
+    return out, kind
 
 
 # ---------------------------------------------------------------------------------------
