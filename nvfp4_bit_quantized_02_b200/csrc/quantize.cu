@@ -8,9 +8,10 @@
 //
 // Two passes over the bf16 input (the tensor scale needs the amax of the whole tensor):
 //   1. amax: 16-byte loads, bf16 magnitudes reduced as packed 16-bit integers (the bf16
-//      magnitude order is the integer order of its low 15 bits), RHT outputs reduced in
-//      fp32; one atomicMax per CTA on the fp32 bit pattern (non-negative floats order like
-//      unsigned ints, and max does not depend on the order of the reduction).
+//      magnitude order is the integer order of its low 15 bits), or in fp32 where the pass
+//      widens the values for the RHT anyway; one atomicMax per CTA on the fp32 bit pattern
+//      (non-negative floats order like unsigned ints, and max does not depend on the order of
+//      the reduction).
 //   2. quantize (quantize_tile_kernel): persistent CTAs take 64 x 256 tiles of x by TMA into
 //      shared memory and emit from one read
 //        - the ROW form (K = columns): a 1x16 block is a lane pair, one shuffle for its amax;
@@ -127,6 +128,8 @@ __global__ void __launch_bounds__(256) amax_plain_kernel(const uint16_t* __restr
 // pass 1b: plain amax and amax of the 16-point RHT along rows (one read).  A thread takes a
 // 16-row x 2-column patch (16 four-byte loads; a warp reads 128 contiguous bytes per row), the
 // column pair transformed as f32x2 pairs.  Few registers per thread keep many patches in flight.
+// The plain amax is a three-input fp32 max over the widened values that propagates NaN (the sign
+// flips do not change magnitudes); the butterfly's final 1/4 is applied once, to the max.
 // rows % 16 == 0, cols % 2 == 0.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
@@ -138,8 +141,7 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
     const int64_t cpr = cols >> 1;
     const int64_t groups = rows >> 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    uint32_t m = 0;
-    float mr = 0.0f;
+    float mp = 0.0f, mr = 0.0f;
     for (GridWalk w((int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride, cpr); w.r < groups; w.next()) {
         const uint16_t* base = x + (w.r << 4) * ld + (w.k << 1);
         uint32_t v[16];
@@ -149,10 +151,23 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
         uint64_t f[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            m = mag_max2(m, v[i]);
             f[i] = bf16x2_to_f2(v[i] ^ sm.m[i]);
+            float a0, a1;
+            f2_split(f[i], a0, a1);
+            asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(mp) : "f"(mp), "f"(fabsf(a0)), "f"(fabsf(a1)));
         }
-        rht16_pairs(f);
+        // the butterfly without its final 1/4: RN(x / 4) is monotonic, so the max of the scaled
+        // outputs is the scaled max
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (i & h) continue;
+                const uint64_t a = f[i], b = f[i + h];
+                f[i] = f2_add(a, b);
+                f[i + h] = f2_sub(a, b);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
             float a0, a1, b0, b1;
@@ -161,9 +176,9 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
             mr = max3_abs(max3_abs(mr, a0, a1), b0, b1);
         }
     }
-    uint32_t mag = max(m & 0xFFFFu, m >> 16);
-    if (mag >= 0x7F80u || !(mr < __int_as_float(0x7F800000))) atomicOr(flags, kFlagNonFinite);
-    block_atomic_max(mag << 16, amax_plain_bits, red);
+    mr = __fmul_rn(mr, 0.25f);
+    if (!(mp < __int_as_float(0x7F800000)) || !(mr < __int_as_float(0x7F800000))) atomicOr(flags, kFlagNonFinite);
+    block_atomic_max(__float_as_uint(mp), amax_plain_bits, red);
     block_atomic_max(__float_as_uint(mr), amax_rht_bits, red);
 }
 
@@ -194,7 +209,10 @@ constexpr int kTileRows = 64;
 constexpr int kTileCols = 256;
 constexpr int kQuantThreads = 256;
 constexpr int kTileBytes = kTileRows * kTileCols * 2;        // 32 KiB of bf16
-constexpr int kStageCodeBytes = 4 * kTileCols * 8;           // [group][column] x 8 bytes
+// [group][column] x 8 bytes, each group padded by 32 bytes: the S phase's lanes read two groups at
+// once (2 apart), which then sit 64 bytes apart in the banks instead of on the same ones
+constexpr int kCodeGroupBytes = kTileCols * 8 + 32;
+constexpr int kStageCodeBytes = 4 * kCodeGroupBytes;
 constexpr int kStageScaleBytes = 4 * kTileCols;              // [group][column]
 
 struct QuantSmem {
@@ -356,19 +374,25 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
 
         // ---- T: 16x16 tile scales ------------------------------------------------------------
         if (b16) {
-            const int tile = tid >> 2, q = tid & 3;          // 64 tiles: 4 row groups x 16 column groups
-            const int g = tile >> 4, cg = tile & 15;
+            // lane = (row quarter q, tile cgl of the warp's 8): the 8 lanes of a quarter-warp read 8
+            // different 16-byte bank groups (lanes 4..7 of each group read their second half first)
+            const int lane = tid & 31, wq = tid >> 5;
+            const int cgl = lane & 7, q = lane >> 3;
+            const int g = wq >> 1, cg = ((wq & 1) << 3) + cgl;
+            const int tile = (g << 4) + cg;
+            const int hf = (cgl >> 2) & 1;
             uint32_t m = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint4* rowp = reinterpret_cast<const uint4*>(sx + (g * 16 + q * 4 + i) * kTileCols + cg * 16);
-                const uint4 a = rowp[0], b = rowp[1];
+                const uint16_t* rowp = sx + (g * 16 + q * 4 + i) * kTileCols + cg * 16;
+                const uint4 a = *reinterpret_cast<const uint4*>(rowp + 8 * hf);
+                const uint4 b = *reinterpret_cast<const uint4*>(rowp + 8 * (hf ^ 1));
                 m = mag_max2(m, a.x); m = mag_max2(m, a.y); m = mag_max2(m, a.z); m = mag_max2(m, a.w);
                 m = mag_max2(m, b.x); m = mag_max2(m, b.y); m = mag_max2(m, b.z); m = mag_max2(m, b.w);
             }
             m = max(m & 0xFFFFu, m >> 16);
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
             const uint32_t code = e4m3_of_amax(__uint_as_float(m << 16), ROW ? senc_r : senc_c);
             if (q == 0) {
                 s_tile_code[tile] = (uint8_t)code;
@@ -390,8 +414,12 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
             for (int j = tid; j < kTileRows * (kTileCols / 16); j += kQuantThreads) {
                 const int r = j >> 4, b = j & 15;
                 const int64_t gr = r_base + r, gc = c_base + b * 16;
-                const uint4 v0 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16);
-                const uint4 v1 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16 + 8);
+                // without SR, lanes with (b >> 2) odd read their block's second half first, so that the
+                // 8 lanes of a quarter-warp hit 8 different 16-byte bank groups; the two code words are
+                // put back in order at the store (under SR the swap costs more than it saves)
+                const int hf = SR ? 0 : (b >> 2) & 1;
+                const uint4 v0 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16 + 8 * hf);
+                const uint4 v1 = *reinterpret_cast<const uint4*>(sx + r * kTileCols + b * 16 + 8 * (hf ^ 1));
                 const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                 uint32_t code;
                 float mult;
@@ -430,8 +458,9 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                 uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
                 sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
                 if (gr < rows && gc < cols) {
+                    const uint32_t c0 = pack4(byte[0], byte[1], byte[2], byte[3]), c1 = pack4(byte[4], byte[5], byte[6], byte[7]);
                     *reinterpret_cast<uint2*>(p.codes_row + gr * (cols >> 1) + (gc >> 1)) =
-                        make_uint2(pack4(byte[0], byte[1], byte[2], byte[3]), pack4(byte[4], byte[5], byte[6], byte[7]));
+                        make_uint2(hf ? c1 : c0, hf ? c0 : c1);
                     if ((b & 3) == 0) {
                         // blocks past `cols` are padding and must read 0
                         const int64_t kb = gc >> 4;
@@ -519,7 +548,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     out[3] = pack4(bc1[4], bc1[5], bc1[6], bc1[7]);
                 }
                 const bool grp_ok = r_base + g * 16 < rows;
-                *reinterpret_cast<uint4*>(s_codes + (g * kTileCols + c) * 8) = make_uint4(out[0], out[1], out[2], out[3]);
+                *reinterpret_cast<uint4*>(s_codes + g * kCodeGroupBytes + c * 8) = make_uint4(out[0], out[1], out[2], out[3]);
                 *reinterpret_cast<uint16_t*>(s_scales + g * kTileCols + c) = grp_ok ? (uint16_t)(code0 | (code1 << 8)) : (uint16_t)0;
             }
             __syncthreads();
@@ -532,8 +561,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                 for (int j = tid; j < 2 * kTileCols; j += kQuantThreads) {
                     const int c = j >> 1, half = j & 1;
                     if (c_base + c < cols && 2 * half < ngroups) {
-                        const uint2 lo = *reinterpret_cast<const uint2*>(s_codes + ((2 * half) * kTileCols + c) * 8);
-                        const uint2 hi = *reinterpret_cast<const uint2*>(s_codes + ((2 * half + 1) * kTileCols + c) * 8);
+                        const uint2 lo = *reinterpret_cast<const uint2*>(s_codes + (2 * half) * kCodeGroupBytes + c * 8);
+                        const uint2 hi = *reinterpret_cast<const uint2*>(s_codes + (2 * half + 1) * kCodeGroupBytes + c * 8);
                         *reinterpret_cast<uint4*>(p.codes_col + (c_base + c) * kbytes + (r_base >> 1) + half * 16) =
                             make_uint4(lo.x, lo.y, hi.x, hi.y);
                     }
@@ -544,7 +573,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     const int c = j >> 2, g = j & 3;
                     if (c_base + c < cols && g < ngroups)
                         *reinterpret_cast<uint2*>(p.codes_col + (c_base + c) * kbytes + (r_base >> 1) + g * 8) =
-                            *reinterpret_cast<const uint2*>(s_codes + (g * kTileCols + c) * 8);
+                            *reinterpret_cast<const uint2*>(s_codes + g * kCodeGroupBytes + c * 8);
                 }
             }
             for (int c = tid; c < kTileCols; c += kQuantThreads) {
