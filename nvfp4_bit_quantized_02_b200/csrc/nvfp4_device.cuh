@@ -86,6 +86,31 @@ __device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
         : "f"(hi), "f"(lo));
     return r;
 }
+// Eight values (four pairs) -> one word of codes, pair q in byte q (first value in the low
+// nibble).  The four conversions write byte registers that one move packs: no widening of each
+// byte and no byte permutes, which the per-pair form above needs to assemble the same word.
+__device__ __forceinline__ uint32_t e2m1x8_word(float a0, float a1, float b0, float b1, float c0, float c1, float d0,
+                                                float d1) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+        "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+        : "=r"(r)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1), "f"(d0), "f"(d1));
+    return r;
+}
+// the same from four f32x2 pairs
+__device__ __forceinline__ uint32_t e2m1x8_word(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3) {
+    float a0, a1, b0, b1, c0, c1, d0, d1;
+    f2_split(p0, a0, a1);
+    f2_split(p1, b0, b1);
+    f2_split(p2, c0, c1);
+    f2_split(p3, d0, d1);
+    return e2m1x8_word(a0, a1, b0, b1, c0, c1, d0, d1);
+}
 
 // ---------------------------------------------------------------------------------------
 // E2M1 stochastic rounding.  For |u| in [lo, hi) of the grid {0,.5,1,1.5,2,3,4,6} the value

@@ -291,10 +291,6 @@ __device__ __forceinline__ U4 sr_words_p(const QuantParams& p, uint32_t stream_i
     return U4{c0, c1, c2, c3};
 }
 
-// four code bytes (each in the low 8 bits of its word) -> one word, byte 0 first
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-}
 
 template <bool ROW, bool COL, bool SR>
 __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx,
@@ -436,7 +432,6 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     mult = s_mult_row[code];
                 }
                 const uint64_t mm = f2(mult, mult);
-                uint32_t byte[8];
                 uint64_t uv[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) uv[q] = f2_mul(bf16x2_to_f2(w[q]), mm);
@@ -449,16 +444,10 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     for (int q = 0; q < 8; ++q)
                         uv[q] = e2m1_sr_values(uv[q], sr_field_bits(rr[q], false), sr_field_bits(rr[q], true));
                 }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float lo, hi;
-                    f2_split(uv[q], lo, hi);
-                    byte[q] = e2m1x2_rne(lo, hi);
-                }
                 uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
                 sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
                 if (gr < rows && gc < cols) {
-                    const uint32_t c0 = pack4(byte[0], byte[1], byte[2], byte[3]), c1 = pack4(byte[4], byte[5], byte[6], byte[7]);
+                    const uint32_t c0 = e2m1x8_word(uv[0], uv[1], uv[2], uv[3]), c1 = e2m1x8_word(uv[4], uv[5], uv[6], uv[7]);
                     *reinterpret_cast<uint2*>(p.codes_row + gr * (cols >> 1) + (gc >> 1)) =
                         make_uint2(hf ? c1 : c0, hf ? c0 : c1);
                     if ((b & 3) == 0) {
@@ -533,19 +522,13 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     }
                 }
                 {
-                    uint32_t bc0[8], bc1[8];
+                    float e0[16], e1[16];   // column c and column c + 1, rows 0..15
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float a0, a1, b0, b1;
-                        f2_split(v[2 * q], a0, a1);
-                        f2_split(v[2 * q + 1], b0, b1);
-                        bc0[q] = e2m1x2_rne(a0, b0);
-                        bc1[q] = e2m1x2_rne(a1, b1);
-                    }
-                    out[0] = pack4(bc0[0], bc0[1], bc0[2], bc0[3]);
-                    out[1] = pack4(bc0[4], bc0[5], bc0[6], bc0[7]);
-                    out[2] = pack4(bc1[0], bc1[1], bc1[2], bc1[3]);
-                    out[3] = pack4(bc1[4], bc1[5], bc1[6], bc1[7]);
+                    for (int i = 0; i < 16; ++i) f2_split(v[i], e0[i], e1[i]);
+                    out[0] = e2m1x8_word(e0[0], e0[1], e0[2], e0[3], e0[4], e0[5], e0[6], e0[7]);
+                    out[1] = e2m1x8_word(e0[8], e0[9], e0[10], e0[11], e0[12], e0[13], e0[14], e0[15]);
+                    out[2] = e2m1x8_word(e1[0], e1[1], e1[2], e1[3], e1[4], e1[5], e1[6], e1[7]);
+                    out[3] = e2m1x8_word(e1[8], e1[9], e1[10], e1[11], e1[12], e1[13], e1[14], e1[15]);
                 }
                 const bool grp_ok = r_base + g * 16 < rows;
                 *reinterpret_cast<uint4*>(s_codes + g * kCodeGroupBytes + c * 8) = make_uint4(out[0], out[1], out[2], out[3]);
@@ -693,7 +676,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                 const uint32_t code = ue8m0_of_mag(max(m & 0xFFFFu, m >> 16));
                 const float inv = ue8m0_inv(code);
                 const uint64_t mm = f2(inv, inv);
-                uint32_t byte[16];
+                uint64_t uv[16];   // the 16 pairs after scaling (and SR onto the grid)
                 if (p.sr) {
                     const uint64_t g0 = ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3;
 #pragma unroll
@@ -701,28 +684,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                         const U4 rw = mx_words(p, g0 + c);
                         const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float lo, hi;
-                            f2_split(e2m1_sr_values(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), sr_field_bits(rr[q], false),
-                                                    sr_field_bits(rr[q], true)),
-                                     lo, hi);
-                            byte[4 * c + q] = e2m1x2_rne(lo, hi);
-                        }
+                        for (int q = 0; q < 4; ++q)
+                            uv[4 * c + q] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), sr_field_bits(rr[q], false),
+                                                           sr_field_bits(rr[q], true));
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        float lo, hi;
-                        f2_split(f2_mul(bf16x2_to_f2(w[q]), mm), lo, hi);
-                        byte[q] = e2m1x2_rne(lo, hi);
-                    }
+                    for (int q = 0; q < 16; ++q) uv[q] = f2_mul(bf16x2_to_f2(w[q]), mm);
                 }
                 uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
                 sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
                 if (gr < rows && gc < cols) {
                     *reinterpret_cast<uint4*>(p.codes + gr * (cols >> 1) + (gc >> 1)) =
-                        make_uint4(pack4(byte[0], byte[1], byte[2], byte[3]), pack4(byte[4], byte[5], byte[6], byte[7]),
-                                   pack4(byte[8], byte[9], byte[10], byte[11]), pack4(byte[12], byte[13], byte[14], byte[15]));
+                        make_uint4(e2m1x8_word(uv[0], uv[1], uv[2], uv[3]), e2m1x8_word(uv[4], uv[5], uv[6], uv[7]),
+                                   e2m1x8_word(uv[8], uv[9], uv[10], uv[11]), e2m1x8_word(uv[12], uv[13], uv[14], uv[15]));
                     if ((b & 3) == 0) {
                         const int64_t kb = gc >> 5;
                         const int64_t nv64 = (cols >> 5) - kb;
@@ -759,32 +734,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                         for (int i = 0; i < 8; ++i)
                             sv[i] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), sr_field_bits(ra[i >> 1], i & 1),
                                                    sr_field_bits(rb[i >> 1], i & 1));
-                        uint32_t b0[4], b1[4];
+                        float e0[8], e1[8];   // column c and column c + 1, rows 8h .. 8h + 7
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float a0, a1, c0v, c1v;
-                            f2_split(sv[2 * q], a0, a1);
-                            f2_split(sv[2 * q + 1], c0v, c1v);
-                            b0[q] = e2m1x2_rne(a0, c0v);
-                            b1[q] = e2m1x2_rne(a1, c1v);
-                        }
-                        out[h] = pack4(b0[0], b0[1], b0[2], b0[3]);
-                        out[4 + h] = pack4(b1[0], b1[1], b1[2], b1[3]);
+                        for (int i = 0; i < 8; ++i) f2_split(sv[i], e0[i], e1[i]);
+                        out[h] = e2m1x8_word(e0[0], e0[1], e0[2], e0[3], e0[4], e0[5], e0[6], e0[7]);
+                        out[4 + h] = e2m1x8_word(e1[0], e1[1], e1[2], e1[3], e1[4], e1[5], e1[6], e1[7]);
                     }
                 } else {
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        uint32_t b0[4], b1[4];
+                        float e0[8], e1[8];   // column c and column c + 1, rows 8h .. 8h + 7
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float a0, a1, c0v, c1v;
-                            f2_split(f2_mul(bf16x2_to_f2(w[8 * h + 2 * q]), mm), a0, a1);
-                            f2_split(f2_mul(bf16x2_to_f2(w[8 * h + 2 * q + 1]), mm), c0v, c1v);
-                            b0[q] = e2m1x2_rne(a0, c0v);
-                            b1[q] = e2m1x2_rne(a1, c1v);
-                        }
-                        out[h] = pack4(b0[0], b0[1], b0[2], b0[3]);
-                        out[4 + h] = pack4(b1[0], b1[1], b1[2], b1[3]);
+                        for (int i = 0; i < 8; ++i) f2_split(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), e0[i], e1[i]);
+                        out[h] = e2m1x8_word(e0[0], e0[1], e0[2], e0[3], e0[4], e0[5], e0[6], e0[7]);
+                        out[4 + h] = e2m1x8_word(e1[0], e1[1], e1[2], e1[3], e1[4], e1[5], e1[6], e1[7]);
                     }
                 }
                 const bool grp_ok = r_base + g * 32 < rows;
@@ -870,7 +833,7 @@ cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int
                               uint32_t* flags, cudaStream_t s) {
     const int64_t chunks = rows * (cols >> 3);
     if (chunks == 0) return cudaSuccess;
-    amax_plain_kernel<<<grid_for(chunks, 256, 8), 256, 0, s>>>(x, rows, cols, ld, amax, flags);
+    amax_plain_kernel<<<grid_for(chunks, 256, 4), 256, 0, s>>>(x, rows, cols, ld, amax, flags);
     return cudaGetLastError();
 }
 

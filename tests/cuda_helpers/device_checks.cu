@@ -17,6 +17,13 @@ __global__ void k_e2m1_rne(uint32_t start, int64_t n, uint8_t* out) {
         out[i] = (uint8_t)e2m1x2_rne(x, x);
     }
 }
+// eight values per word, as the quantize kernels pack them: out[i] = codes of x[8i .. 8i + 7]
+__global__ void k_e2m1x8(const float* x, int64_t nwords, uint32_t* out) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nwords; i += (int64_t)gridDim.x * blockDim.x) {
+        const float* v = x + 8 * i;
+        out[i] = e2m1x8_word(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    }
+}
 __global__ void k_e2m1_sr_threshold(uint32_t start, int64_t n, uint32_t* out) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         out[i] = e2m1_sr_threshold((start + (uint32_t)i) & 0x7FFFFFFFu);
@@ -71,6 +78,7 @@ static int grid(int64_t n) { int64_t g = (n + 255) / 256; return (int)(g < 4096 
 
 extern "C" {
 int chk_e2m1_rne(uint32_t start, int64_t n, uint8_t* out) { k_e2m1_rne<<<grid(n), 256>>>(start, n, out); return (int)cudaDeviceSynchronize(); }
+int chk_e2m1x8(const float* x, int64_t nwords, uint32_t* out) { k_e2m1x8<<<grid(nwords), 256>>>(x, nwords, out); return (int)cudaDeviceSynchronize(); }
 int chk_e2m1_sr_threshold(uint32_t start, int64_t n, uint32_t* out) { k_e2m1_sr_threshold<<<grid(n), 256>>>(start, n, out); return (int)cudaDeviceSynchronize(); }
 int chk_e2m1_sr(const float* x, const uint32_t* r, int64_t n, uint8_t* out) { k_e2m1_sr<<<grid(n), 256>>>(x, r, n, out); return (int)cudaDeviceSynchronize(); }
 int chk_e4m3(uint32_t start, int64_t n, uint8_t* out) { k_e4m3<<<grid(n), 256>>>(start, n, out); return (int)cudaDeviceSynchronize(); }

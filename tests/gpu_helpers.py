@@ -131,6 +131,7 @@ def checks():
         L = ctypes.CDLL(mod.build())
         vp, i64, u32, u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
         L.chk_e2m1_rne.argtypes = [u32, i64, vp]
+        L.chk_e2m1x8.argtypes = [vp, i64, vp]
         L.chk_e2m1_sr_threshold.argtypes = [u32, i64, vp]
         L.chk_e2m1_sr.argtypes = [vp, vp, i64, vp]
         L.chk_e4m3.argtypes = [u32, i64, vp]

@@ -45,6 +45,30 @@ def test_e2m1_rne_all_finite_fp32():
         _sweep(lo, hi, L.chk_e2m1_rne, oracle.e2m1_rne, np.uint8, torch.uint8, transform=both)
 
 
+def test_e2m1_eight_per_word_packing():
+    # the quantize kernels convert eight values into one code word (byte q = pair q, first value
+    # in the low nibble): every nibble position against the oracle's RNE code of its value, over
+    # random fp32 bit patterns and the grid's ties, values and neighbours in every position
+    L = checks()
+    rng = np.random.default_rng(8)
+    grid = np.array([0, .25, .5, .75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 7, 1e30, np.inf, np.nan], np.float32)
+    near = np.concatenate([np.nextafter(grid, np.float32(np.inf)), np.nextafter(grid, np.float32(-np.inf))])
+    special = np.concatenate([grid, -grid, near, -near])
+    special = np.concatenate([np.roll(special, k) for k in range(8)])   # each value in every nibble position
+    x = np.concatenate([rng.integers(0, 1 << 32, 1 << 22, dtype=np.uint64).astype(np.uint32).view(np.float32),
+                        special])
+    x = np.concatenate([x, np.zeros(-x.size % 8, np.float32)])
+    xd = torch.from_numpy(x).cuda()
+    out = torch.empty(x.size // 8, dtype=torch.int32, device="cuda")
+    assert L.chk_e2m1x8(ctypes.c_void_p(xd.data_ptr()), x.size // 8, ctypes.c_void_p(out.data_ptr())) == 0
+    b = out.cpu().numpy().view(np.uint8)                         # little-endian: byte q of word i at 4i + q
+    got = np.stack([b & 15, b >> 4], axis=1).reshape(-1)         # low nibble first
+    finite = np.isfinite(x)
+    want = np.zeros(x.size, np.uint8)
+    want[finite] = oracle.e2m1_rne(x[finite])
+    assert np.array_equal(got[finite], want[finite])
+
+
 def test_e2m1_sr_threshold_all_below_six():
     L = checks()
     _sweep(0x00000000, 0x40C00000, L.chk_e2m1_sr_threshold, oracle.e2m1_sr_threshold, np.uint32, torch.int32,
