@@ -841,7 +841,7 @@ cudaError_t launch_amax_rht(const uint16_t* x, int64_t rows, int64_t cols, int64
                             uint32_t* amax_plain, uint32_t* amax_rht, uint32_t* flags, cudaStream_t s) {
     const int64_t units = (rows >> 4) * (cols >> 1);
     if (units == 0) return cudaSuccess;
-    amax_rht_kernel<<<grid_for(units, 256, 8), 256, 0, s>>>(x, rows, cols, ld, sign_masks(signs), amax_plain,
+    amax_rht_kernel<<<grid_for(units, 256, 4), 256, 0, s>>>(x, rows, cols, ld, sign_masks(signs), amax_plain,
                                                            amax_rht, flags);
     return cudaGetLastError();
 }
