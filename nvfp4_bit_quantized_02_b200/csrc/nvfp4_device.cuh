@@ -140,19 +140,24 @@ __device__ __forceinline__ uint32_t e2m1_sr_threshold(uint32_t a /* |u| bits */)
 //     of 1.5 s 2^23 that follows is exact.
 // The result is a signed grid value (the sign of u, also for a zero result), 8 where |u| > 6
 // rounded up: the hardware RNE conversion to E2M1 then encodes it exactly (8 saturates to 6).
-// rb_lo / rb_hi are the fp32 bits of 2^23 + r16 (sr_field_bits).
-__device__ __forceinline__ uint32_t sr_field_bits(uint32_t word, bool high) {
-    // 2^23 + the low (high = false) or the high 16-bit field of a Philox word, as fp32 bits
-    return __byte_perm(word, 0x4B000000u, high ? 0x7432u : 0x7410u);
+// r_lo / r_hi are the elements' 16-bit fields r16 as fp32 numbers (exact; sr_field).
+__device__ __forceinline__ float sr_field(uint32_t word, bool high) {
+    // the low (high = false) or the high 16-bit field of a Philox word, converted to fp32 by the
+    // integer-to-float unit (which the encode's other instructions leave idle)
+    float r;
+    if (high)
+        asm("{\n\t.reg .u16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.rn.f32.u16 %0, b;\n\t}" : "=f"(r) : "r"(word));
+    else
+        asm("{\n\t.reg .u16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.rn.f32.u16 %0, a;\n\t}" : "=f"(r) : "r"(word));
+    return r;
 }
-__device__ __forceinline__ uint64_t e2m1_sr_values(uint64_t u, uint32_t rb_lo, uint32_t rb_hi) {
+__device__ __forceinline__ uint64_t e2m1_sr_values(uint64_t u, float r_lo, float r_hi) {
     float ul, uh;
     f2_split(u, ul, uh);
     const float el = fmaxf(__uint_as_float(__float_as_uint(ul) & 0x7F800000u), 1.0f);   // 2^max(e, 0)
     const float eh = fmaxf(__uint_as_float(__float_as_uint(uh) & 0x7F800000u), 1.0f);
     const uint64_t nsq = f2_mul(f2(el, eh), f2c(-0x1p-17f));                              // -s / 2^16
-    const uint64_t r = f2_sub(f2(__uint_as_float(rb_lo), __uint_as_float(rb_hi)), f2c(8388608.0f));   // r16
-    const uint64_t w = f2_fma(nsq, r, f2(fabsf(ul), fabsf(uh)));
+    const uint64_t w = f2_fma(nsq, f2(r_lo, r_hi), f2(fabsf(ul), fabsf(uh)));
     const uint64_t m = f2_mul(nsq, f2c(-0x1.8p+39f));                                     // 1.5 s 2^23
     uint64_t t;
     asm("add.rp.f32x2 %0, %1, %2;" : "=l"(t) : "l"(w), "l"(m));
@@ -162,9 +167,9 @@ __device__ __forceinline__ uint64_t e2m1_sr_values(uint64_t u, uint32_t rb_lo, u
 }
 // One element: its code in bits [0, 4)
 __device__ __forceinline__ uint32_t e2m1_sr(float u, uint32_t r16) {
-    const uint32_t rb = 0x4B000000u | (r16 & 0xFFFFu);
+    const float r = sr_field(r16, false);
     float vl, vh;
-    f2_split(e2m1_sr_values(f2(u, u), rb, rb), vl, vh);
+    f2_split(e2m1_sr_values(f2(u, u), r, r), vl, vh);
     return e2m1x2_rne(vl, vh) & 15u;
 }
 

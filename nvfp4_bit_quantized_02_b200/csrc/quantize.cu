@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                     const uint32_t rr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        uv[q] = e2m1_sr_values(uv[q], sr_field_bits(rr[q], false), sr_field_bits(rr[q], true));
+                        uv[q] = e2m1_sr_values(uv[q], sr_field(rr[q], false), sr_field(rr[q], true));
                 }
                 uint32_t sw = code | (__shfl_down_sync(0xFFFFFFFFu, code, 1) << 8);
                 sw |= __shfl_down_sync(0xFFFFFFFFu, sw, 2) << 16;
@@ -517,8 +517,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
                         const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            v[8 * h + i] = e2m1_sr_values(v[8 * h + i], sr_field_bits(ra[i >> 1], i & 1),
-                                                          sr_field_bits(rb[i >> 1], i & 1));
+                            v[8 * h + i] = e2m1_sr_values(v[8 * h + i], sr_field(ra[i >> 1], i & 1),
+                                                          sr_field(rb[i >> 1], i & 1));
                     }
                 }
                 {
@@ -685,8 +685,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                         const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            uv[4 * c + q] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), sr_field_bits(rr[q], false),
-                                                           sr_field_bits(rr[q], true));
+                            uv[4 * c + q] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[4 * c + q]), mm), sr_field(rr[q], false),
+                                                           sr_field(rr[q], true));
                     }
                 } else {
 #pragma unroll
@@ -732,8 +732,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                         uint64_t sv[8];   // row i: the SR values of columns c and c + 1
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            sv[i] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), sr_field_bits(ra[i >> 1], i & 1),
-                                                   sr_field_bits(rb[i >> 1], i & 1));
+                            sv[i] = e2m1_sr_values(f2_mul(bf16x2_to_f2(w[8 * h + i]), mm), sr_field(ra[i >> 1], i & 1),
+                                                   sr_field(rb[i >> 1], i & 1));
                         float e0[8], e1[8];   // column c and column c + 1, rows 8h .. 8h + 7
 #pragma unroll
                         for (int i = 0; i < 8; ++i) f2_split(sv[i], e0[i], e1[i]);
