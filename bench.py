@@ -41,17 +41,25 @@ FP4_DENSE_DATASHEET_TFLOPS = 9000.0
 # this GPU: four 128x256x64 MMAs take 512 cycles), 148 SMs
 FP4_FLOP_PER_CLK = 2 * 16384 * 148
 # DRAM bytes (read + write) per GEMM launch, the mean over the fprop, dgrad and wgrad launches
-# of one ncu capture of the SM-pair GEMM at this layer's shapes, valid for the GEMM source it was
-# taken on only: reported as null once gemm_sm100.cu no longer hashes to that source.
-GEMM_SRC = os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", "gemm_sm100.cu")
-GEMM_TRAFFIC = {"sha256": "555920f7094baece1d9230ea0c01e6ca2a9928cb999f4e326352c9f16d6b5248",
-                "bytes_per_launch": 483.7e6}
+# of one ncu capture of the SM-pair GEMM at this layer's shapes, valid for the GEMM sources it was
+# taken on only (the kernel file and the device header it includes): reported as null once they
+# no longer hash to those sources.
+GEMM_SRCS = [os.path.join(ROOT, "nvfp4_bit_quantized_02_b200", "csrc", f) for f in ("gemm_sm100.cu", "nvfp4_device.cuh")]
+GEMM_TRAFFIC = {"sha256": "2d68f32034fdb4cd69f13713f8e15c3a40a64b119d1956d1ee305df8c54f9192",
+                "bytes_per_launch": 478.2e6}
+
+
+def gemm_src_hash():
+    h = hashlib.sha256()
+    for path in GEMM_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def gemm_traffic():
     try:
-        with open(GEMM_SRC, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
+        h = gemm_src_hash()
     except OSError:
         return None
     return GEMM_TRAFFIC["bytes_per_launch"] if h == GEMM_TRAFFIC["sha256"] else None
