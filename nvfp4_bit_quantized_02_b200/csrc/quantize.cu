@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "nvfp4_device.cuh"
@@ -819,10 +820,41 @@ __global__ void __launch_bounds__(256) transpose_2d_kernel(const uint8_t* __rest
 // ---------------------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------------------
+// SM count of the current device, looked up once per device
+static int q_sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+// Resident CTAs per SM of a tile kernel on the current device, with its dynamic shared-memory
+// limit raised first; both are per-device facts of the kernel, established once per device
+// (`cache` belongs to one kernel instantiation).  0 on a CUDA error.
+template <typename Kernel>
+static int tile_ctas_per_sm(Kernel kern, int threads, int smem, std::atomic<int> (&cache)[64]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const bool cacheable = dev >= 0 && dev < 64;
+    if (cacheable) {
+        const int n = cache[dev].load(std::memory_order_acquire);
+        if (n > 0) return n;
+    }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
+    if (per_sm < 1) per_sm = 1;
+    if (cacheable) cache[dev].store(per_sm, std::memory_order_release);
+    return per_sm;
+}
+
 static int grid_for(int64_t work_items, int threads, int per_sm) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = q_sm_count();
     int64_t want = (work_items + threads - 1) / threads;
     int64_t cap = (int64_t)sms * per_sm;
     if (want < 1) want = 1;
@@ -890,14 +922,14 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
                                                                        : quantize_tile_kernel<false, true, true>)
            : (row && col ? quantize_tile_kernel<true, true, false> : row ? quantize_tile_kernel<true, false, false>
                                                                         : quantize_tile_kernel<false, true, false>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantThreads, smem);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t cap = (int64_t)sms * per_sm;
+    static std::atomic<int> cache[6][64];   // one per instantiation: (row, col, sr)
+    const int which = (sr ? 3 : 0) + (row && col ? 0 : row ? 1 : 2);
+    const int per_sm = tile_ctas_per_sm(kern, kQuantThreads, smem, cache[which]);
+    if (per_sm < 1) {
+        const cudaError_t e = cudaGetLastError();
+        return e != cudaSuccess ? e : cudaErrorInvalidValue;
+    }
+    const int64_t cap = (int64_t)q_sm_count() * per_sm;
     const int grid = (int)(ntiles < cap ? ntiles : cap);
     kern<<<grid, kQuantThreads, smem, s>>>(map, q);
     return cudaGetLastError();
@@ -926,14 +958,13 @@ cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_
         k1 += 0xBB67AE85u;
     }
     void (*kern)(const CUtensorMap, const MxParams) = column_form ? quantize_mx_kernel<true> : quantize_mx_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem::bytes);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantThreads, QuantSmem::bytes);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t cap = (int64_t)sms * per_sm;
+    static std::atomic<int> cache[2][64];   // row form, column form
+    const int per_sm = tile_ctas_per_sm(kern, kQuantThreads, QuantSmem::bytes, cache[column_form ? 1 : 0]);
+    if (per_sm < 1) {
+        const cudaError_t e = cudaGetLastError();
+        return e != cudaSuccess ? e : cudaErrorInvalidValue;
+    }
+    const int64_t cap = (int64_t)q_sm_count() * per_sm;
     kern<<<(int)(ntiles < cap ? ntiles : cap), kQuantThreads, QuantSmem::bytes, s>>>(map, q);
     return cudaGetLastError();
 }
