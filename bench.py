@@ -593,8 +593,8 @@ def time_calls(calls, steps, warmup, flush):
 
 
 def variant_fields(args, dev, flush, x, w, dy) -> dict:
-    """The same layer step in the pages' comparison format (MXFP4: six single-pass quantizes and
-    three kind::mxf4 GEMMs) and on the BF16 path of the high-precision layers (three kind::f16
+    """The same layer step in the pages' comparison format (MXFP4: three single-pass quantizes, each
+    giving both forms from one read, and three kind::mxf4 GEMMs) and on the BF16 path of the high-precision layers (three kind::f16
     GEMMs and the transposes of their K-major operands)."""
     import nvfp4_bit_quantized_02_b200 as nv
     ws = nv.Workspace(dev)
@@ -604,13 +604,12 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
     y = torch.empty((T_TOK, D_OUT), dtype=torch.bfloat16, device=dev)
     dx = torch.empty((T_TOK, D_IN), dtype=torch.bfloat16, device=dev)
     dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
-    mq = nv.nvfp4_mx_quantize
+    mq = nv.nvfp4_mx_quantize_dual
     mx_calls = [
-        ("quantize X (row, column)", lambda k: (mq(x, 0, out=f["xr"], ws=ws), mq(x, 1, out=f["xc"], ws=ws))),
-        ("quantize W (row, column)", lambda k: (mq(w, 0, out=f["wr"], ws=ws), mq(w, 1, out=f["wc"], ws=ws))),
+        ("quantize X (row, column)", lambda k: mq(x, out_row=f["xr"], out_col=f["xc"], ws=ws)),
+        ("quantize W (row, column)", lambda k: mq(w, out_row=f["wr"], out_col=f["wc"], ws=ws)),
         ("fprop", lambda k: nv.nvfp4_mx_gemm(f["xr"], f["wr"], out=y, ws=ws)),
-        ("quantize dY (row, column; SR)", lambda k: (mq(dy, 0, nv.SR, k, 1, out=f["dyr"], ws=ws),
-                                                     mq(dy, 1, nv.SR, k, 2, out=f["dyc"], ws=ws))),
+        ("quantize dY (row, column; SR)", lambda k: mq(dy, nv.SR, k, 1, 2, out_row=f["dyr"], out_col=f["dyc"], ws=ws)),
         ("dgrad", lambda k: nv.nvfp4_mx_gemm(f["dyr"], f["wc"], out=dx, ws=ws)),
         ("wgrad", lambda k: nv.nvfp4_mx_gemm(f["dyc"], f["xc"], out=dw, ws=ws)),
     ]
@@ -619,7 +618,7 @@ def variant_fields(args, dev, flush, x, w, dy) -> dict:
         "value": FLOP_STEP / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms, "per_call_ms": per,
         "gemm_tflops": {g: FLOP_GEMM / per[g] / 1e9 for g in ("fprop", "dgrad", "wgrad")},
         "workload": "the same layer with MXFP4 operands (blocks of 32, UE8M0 scales, no tensor scale): X, W and "
-                    "dY each quantized in both forms (dY with SR), three kind::mxf4 GEMMs"}}
+                    "dY each quantized in both forms from one read (dY with SR), three kind::mxf4 GEMMs"}}
     del f
     lay = nv.LinearBF16(T_TOK, D_IN, D_OUT, device=dev)
     bf_calls = [("fwd", lambda k: lay.fwd(x, w, y)), ("bwd", lambda k: lay.bwd(x, w, dy, dx, dw))]

@@ -308,7 +308,8 @@ nvfp4_status nvfp4_poll_noalloc(nvfp4_stream_t stream);
 /*
  * MXFP4, the format the pages compare NVFP4 against (gist.science 2.A: blocks of 32 elements with
  * a power-of-two UE8M0 scale and no tensor scale; 4 "Ergebnisse": MXFP4 needs about 36 % more
- * training tokens to match NVFP4).  One form per call, a single pass (no tensor amax):
+ * training tokens to match NVFP4).  One form per call (nvfp4_mx_quantize) or both forms from one
+ * read (nvfp4_mx_quantize_dual), a single pass (no tensor amax):
  *   scale code of a block = floor(log2 amax_b) - 2 + 127 clamped to [0, 254] (0 for an all-zero
  *   block), i.e. 2^E with E the block's exponent less that of E2M1's largest value (6 = 1.5 * 2^2);
  *   element u = v * 2^-E, encoded to E2M1 as in nvfp4_quantize (RNE, or SR with the same Philox
@@ -331,6 +332,14 @@ size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k); /* ceil(rows/128)*128 * c
 nvfp4_status nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along,
                                nvfp4_round mode, uint64_t sr_seed, uint32_t stream_id,
                                nvfp4_mx_tensor* out, void* ws, nvfp4_stream_t stream);
+/* Both MXFP4 forms of x from one read: out_row (along = 0, SR stream stream_row) and out_col
+ * (along = 1, SR stream stream_col), each equal to the form nvfp4_mx_quantize gives with the same
+ * arguments.  rows % 32 == 0 and cols % 32 == 0; the buffers are the caller's, filled on `stream`;
+ * out_row->rows/k and out_col->rows/k are set. */
+nvfp4_status nvfp4_mx_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
+                                    uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
+                                    nvfp4_mx_tensor* out_row, nvfp4_mx_tensor* out_col, void* ws,
+                                    nvfp4_stream_t stream);
 /* D[M][N] = sum_k A[m][k] * B[n][k] over MXFP4 forms with the same k, by the tcgen05
  * kind::mxf4 block-scaled MMA; fp32 accumulation, bf16 or fp32 output.  Shape rules and kernel
  * choice as nvfp4_gemm (K % 32 == 0). */

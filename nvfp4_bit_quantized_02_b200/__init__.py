@@ -98,6 +98,8 @@ def _lib():
             "nvfp4_linear_bf16_fwd": ([vp, vp, vp, i64, i64, i64, vp, vp], i32),
             "nvfp4_linear_bf16_bwd": ([vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
             "nvfp4_mx_quantize": ([vp, i64, i64, i64, i32, i32, u64, u32, c.POINTER(CMXTensor), vp, vp], i32),
+            "nvfp4_mx_quantize_dual": ([vp, i64, i64, i64, i32, u64, u32, u32, c.POINTER(CMXTensor),
+                                        c.POINTER(CMXTensor), vp, vp], i32),
             "nvfp4_mx_gemm": ([c.POINTER(CMXTensor), c.POINTER(CMXTensor), vp, i64, i32, vp, vp], i32),
             "nvfp4_quantize_noalloc": ([vp, i64, i64, i64, i32, i32, i32, i32, u64, u64, u32, T, vp], i32),
             "nvfp4_poll_noalloc": ([vp], i32),
@@ -448,6 +450,21 @@ def nvfp4_mx_quantize(x: torch.Tensor, along: int = 0, mode: int = RNE, sr_seed:
     _check(_lib().nvfp4_mx_quantize(_ptr(x), rows, cols, ld, along, mode, sr_seed, stream_id, ctypes.byref(ct), ws.ptr,
                                     _stream(stream)), "nvfp4_mx_quantize")
     return out
+
+
+def nvfp4_mx_quantize_dual(x: torch.Tensor, mode: int = RNE, sr_seed: int = 0, stream_row: int = 0, stream_col: int = 0,
+                           out_row: MXTensor | None = None, out_col: MXTensor | None = None,
+                           ws: Workspace | None = None, stream=None):
+    """Both MXFP4 forms of x (along 0 and along 1) from one read."""
+    rows, cols, ld = _bf16_2d(x)
+    out_row = out_row or MXTensor.empty(rows, cols, x.device)
+    out_col = out_col or MXTensor.empty(cols, rows, x.device)
+    ws = ws or default_workspace()
+    a, b = out_row.c(), out_col.c()
+    _check(_lib().nvfp4_mx_quantize_dual(_ptr(x), rows, cols, ld, mode, sr_seed, stream_row, stream_col,
+                                         ctypes.byref(a), ctypes.byref(b), ws.ptr, _stream(stream)),
+           "nvfp4_mx_quantize_dual")
+    return out_row, out_col
 
 
 def nvfp4_mx_gemm(a: MXTensor, b: MXTensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,

@@ -537,14 +537,25 @@ size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k) {
     return (size_t)(((rows + 127) / 128) * 128 * ((k + 127) / 128) * 4);
 }
 
+static nvfp4_status check_mx_out(const nvfp4_mx_tensor* out) {
+    if (!out || !out->codes || !out->scales) return NVFP4_ERR_NULL;
+    if (!aligned16(out->codes) || !aligned16(out->scales)) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
+}
+
+// zero a form's scale tiles where the kernel leaves padding unwritten (R or K/32 ragged)
+static cudaError_t clear_mx_padding(const nvfp4_mx_tensor* out, int64_t R, int64_t K, cudaStream_t s) {
+    if ((R & 127) != 0 || ((K >> 5) & 3) != 0) return cudaMemsetAsync(out->scales, 0, nvfp4_mx_scales_bytes(R, K), s);
+    return cudaSuccess;
+}
+
 nvfp4_status nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int along, nvfp4_round mode,
                                uint64_t sr_seed, uint32_t stream_id, nvfp4_mx_tensor* out, void* ws,
                                nvfp4_stream_t stream) {
     if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
     if (along != 0 && along != 1) return NVFP4_ERR_ARG;
     if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
-    if (!out || !out->codes || !out->scales) return NVFP4_ERR_NULL;
-    if (!aligned16(out->codes) || !aligned16(out->scales)) return NVFP4_ERR_ALIGN;
+    if (nvfp4_status st = check_mx_out(out)) return st;
     if (!ws) return NVFP4_ERR_WORKSPACE;
     const int64_t R = along ? cols : rows, K = along ? rows : cols;
     if (K % 32 != 0) return NVFP4_ERR_SHAPE;
@@ -553,21 +564,65 @@ nvfp4_status nvfp4_mx_quantize(const void* x, int64_t rows, int64_t cols, int64_
     out->k = K;
     if (R == 0 || K == 0) return NVFP4_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((R & 127) != 0 || ((K >> 5) & 3) != 0)
-        if (cudaError_t e = cudaMemsetAsync(out->scales, 0, nvfp4_mx_scales_bytes(R, K), s)) return from_cuda(e);
+    if (cudaError_t e = clear_mx_padding(out, R, K, s)) return from_cuda(e);
     MxParams p;
     std::memset(&p, 0, sizeof(p));
     p.x = reinterpret_cast<const uint16_t*>(x);
     p.rows = rows;
     p.cols = cols;
     p.ld = ldx;
-    p.codes = out->codes;
-    p.scales = out->scales;
-    p.nkt = (K + 127) / 128;
+    if (along == 0) {
+        p.codes = out->codes;
+        p.scales = out->scales;
+        p.nkt = (K + 127) / 128;
+        p.stream_id = stream_id;
+    } else {
+        p.codes_col = out->codes;
+        p.scales_col = out->scales;
+        p.nkt_col = (K + 127) / 128;
+        p.stream_col = stream_id;
+    }
     p.sr = mode == NVFP4_SR;
-    p.stream_id = stream_id;
     p.flags = &ws_of(ws)->flags;
-    return from_cuda(launch_quantize_mx(p, along == 1, sr_seed, s));
+    return from_cuda(launch_quantize_mx(p, along == 0, along == 1, sr_seed, s));
+}
+
+nvfp4_status nvfp4_mx_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ldx, nvfp4_round mode,
+                                    uint64_t sr_seed, uint32_t stream_row, uint32_t stream_col,
+                                    nvfp4_mx_tensor* out_row, nvfp4_mx_tensor* out_col, void* ws,
+                                    nvfp4_stream_t stream) {
+    if (nvfp4_status st = check_input(x, rows, cols, ldx)) return st;
+    if (mode != NVFP4_RNE && mode != NVFP4_SR) return NVFP4_ERR_ARG;
+    if (nvfp4_status st = check_mx_out(out_row)) return st;
+    if (nvfp4_status st = check_mx_out(out_col)) return st;
+    if (!ws) return NVFP4_ERR_WORKSPACE;
+    if (rows % 32 != 0 || cols % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (nvfp4_status st = check_device()) return st;
+    out_row->rows = rows;
+    out_row->k = cols;
+    out_col->rows = cols;
+    out_col->k = rows;
+    if (rows == 0 || cols == 0) return NVFP4_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaError_t e = clear_mx_padding(out_row, rows, cols, s)) return from_cuda(e);
+    if (cudaError_t e = clear_mx_padding(out_col, cols, rows, s)) return from_cuda(e);
+    MxParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = reinterpret_cast<const uint16_t*>(x);
+    p.rows = rows;
+    p.cols = cols;
+    p.ld = ldx;
+    p.codes = out_row->codes;
+    p.scales = out_row->scales;
+    p.nkt = (cols + 127) / 128;
+    p.stream_id = stream_row;
+    p.codes_col = out_col->codes;
+    p.scales_col = out_col->scales;
+    p.nkt_col = (rows + 127) / 128;
+    p.stream_col = stream_col;
+    p.sr = mode == NVFP4_SR;
+    p.flags = &ws_of(ws)->flags;
+    return from_cuda(launch_quantize_mx(p, true, true, sr_seed, s));
 }
 
 nvfp4_status nvfp4_mx_gemm(const nvfp4_mx_tensor* a, const nvfp4_mx_tensor* b, void* d, int64_t ldd,

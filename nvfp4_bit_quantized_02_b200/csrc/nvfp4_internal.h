@@ -70,17 +70,22 @@ struct QuantParams {
 struct MxParams {
     const uint16_t* x;
     int64_t rows, cols, ld;    // the bf16 source [rows][ld]
-    uint8_t* codes;            // the form's codes [R][K/2]
-    uint8_t* scales;           // UE8M0 scales in 128x4 tiles
-    int64_t nkt;               // ceil(K / 128): 128x4 scale tiles per 128 form rows
-    int32_t sr;                // 1: stochastic rounding
-    uint32_t stream_id;
+    // the row form (K = cols) and the column form (K = rows); a call fills the forms it launches
+    uint8_t* codes;            // row form's codes [rows][cols/2]
+    uint8_t* scales;           // its UE8M0 scales in 128x4 tiles
+    int64_t nkt;               // ceil(cols / 128): 128x4 scale tiles per 128 form rows
+    uint32_t stream_id;        // its SR stream
+    uint8_t* codes_col;        // column form's codes [cols][rows/2]
+    uint8_t* scales_col;
+    int64_t nkt_col;           // ceil(rows / 128)
+    uint32_t stream_col;
+    int32_t sr;                // 1: stochastic rounding (both forms)
     uint32_t* flags;           // workspace flags (timeout of a tile copy)
     uint32_t key0[10];         // Philox4x32-10 round keys of the SR seed
     uint32_t key1[10];
 };
 
-cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_seed, cudaStream_t s);
+cudaError_t launch_quantize_mx(const MxParams& p, bool row_form, bool column_form, uint64_t sr_seed, cudaStream_t s);
 
 cudaError_t launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* amax,
                               uint32_t* flags, cudaStream_t s);

@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const _
 // amax pass.  Elements u = v * 2^-E (one exact power-of-two product, rounded only if it lands
 // below the normal range) go through the same E2M1 encoders as NVFP4, RNE or SR; SR fields are
 // indexed by the element's position in the form.  The same TMA-fed persistent tile walk as the
-// NVFP4 quantizer, one form per call:
+// NVFP4 quantizer, one form or both forms from one read of each tile:
 //   ROW form: one thread per 1x32 block (four 16-byte shared loads), 16 code bytes per store;
 //   COL form: one thread per (column pair, 32-row group): the 32 bf16 pairs give both columns'
 //             block maxima by packed integer max, then the codes are staged and leave as rows.
@@ -601,8 +601,8 @@ __device__ __forceinline__ float ue8m0_inv(uint32_t code) {
     return __uint_as_float(code == 254u ? 0x00400000u : (254u - code) << 23);
 }
 
-__device__ __forceinline__ U4 mx_words(const MxParams& p, uint64_t g) {
-    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = p.stream_id, c3 = 0u;
+__device__ __forceinline__ U4 mx_words(const MxParams& p, uint32_t stream_id, uint64_t g) {
+    uint32_t c0 = (uint32_t)g, c1 = (uint32_t)(g >> 32), c2 = stream_id, c3 = 0u;
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
         const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
@@ -616,8 +616,8 @@ __device__ __forceinline__ U4 mx_words(const MxParams& p, uint64_t g) {
     return U4{c0, c1, c2, c3};
 }
 
-template <bool COLF>
-__global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __grid_constant__ CUtensorMap tmx,
+template <bool ROWF, bool COLF>
+__global__ void __launch_bounds__(kQuantThreads, 3) quantize_mx_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                       const __grid_constant__ MxParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x;
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
         ++consumed;
         const uint16_t* sx = reinterpret_cast<const uint16_t*>(smem + (buf ? QuantSmem::x1 : QuantSmem::x0));
         const int64_t r_base = tr * kTileRows, c_base = tc * kTileCols;
-        if (!COLF) {
+        if (ROWF) {
             // ---- ROW form: one thread per 1x32 block; lanes 4a..4a+3 hold four blocks of one row
 #pragma unroll 1
             for (int j = tid; j < kTileRows * (kTileCols / 32); j += kQuantThreads) {
@@ -682,7 +682,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                     const uint64_t g0 = ((uint64_t)gr * (uint64_t)cols + (uint64_t)gc) >> 3;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        const U4 rw = mx_words(p, g0 + c);
+                        const U4 rw = mx_words(p, p.stream_id, g0 + c);
                         const uint32_t rr[4] = {rw.x, rw.y, rw.z, rw.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
@@ -708,7 +708,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                     }
                 }
             }
-        } else {
+        }
+        if (COLF) {
             // ---- COL form: one thread per (column pair, 32-row group) -------------------------
             {
                 const int cp = tid & (kTileCols / 2 - 1), g = tid >> 7;
@@ -728,7 +729,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
                     const uint64_t g1 = g0 + ((uint64_t)rows >> 3);
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {   // rows 8h .. 8h + 7: one Philox call per column
-                        const U4 a = mx_words(p, g0 + h), bw = mx_words(p, g1 + h);
+                        const U4 a = mx_words(p, p.stream_col, g0 + h), bw = mx_words(p, p.stream_col, g1 + h);
                         const uint32_t ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {bw.x, bw.y, bw.z, bw.w};
                         uint64_t sv[8];   // row i: the SR values of columns c and c + 1
 #pragma unroll
@@ -765,12 +766,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quantize_mx_kernel(const __g
             for (int j = tid; j < 2 * kTileCols; j += kQuantThreads) {
                 const int c = j >> 1, g = j & 1;
                 if (c_base + c < cols && g < ngroups)
-                    *reinterpret_cast<uint4*>(p.codes + (c_base + c) * kbytes + (r_base >> 1) + g * 16) =
+                    *reinterpret_cast<uint4*>(p.codes_col + (c_base + c) * kbytes + (r_base >> 1) + g * 16) =
                         *reinterpret_cast<const uint4*>(s_codes + (g * kTileCols + c) * 16);
             }
             for (int c = tid; c < kTileCols; c += kQuantThreads) {
                 if (c_base + c < cols) {
-                    uint8_t* dst = p.scales + scale_offset(c_base + c, r_base >> 5, p.nkt);
+                    uint8_t* dst = p.scales_col + scale_offset(c_base + c, r_base >> 5, p.nkt_col);
                     dst[0] = s_scales[c];
                     if (ngroups > 1) dst[1] = s_scales[kTileCols + c];
                 }
@@ -935,7 +936,8 @@ cudaError_t launch_quantize_tiles(const QuantParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_seed, cudaStream_t s) {
+cudaError_t launch_quantize_mx(const MxParams& p, bool row_form, bool column_form, uint64_t sr_seed, cudaStream_t s) {
+    if (!row_form && !column_form) return cudaErrorInvalidValue;
     const int64_t ntiles = ((p.rows + kTileRows - 1) / kTileRows) * ((p.cols + kTileCols - 1) / kTileCols);
     if (ntiles == 0) return cudaSuccess;
     auto fn = q_encode_fn();
@@ -957,9 +959,12 @@ cudaError_t launch_quantize_mx(const MxParams& p, bool column_form, uint64_t sr_
         k0 += 0x9E3779B9u;
         k1 += 0xBB67AE85u;
     }
-    void (*kern)(const CUtensorMap, const MxParams) = column_form ? quantize_mx_kernel<true> : quantize_mx_kernel<false>;
-    static std::atomic<int> cache[2][64];   // row form, column form
-    const int per_sm = tile_ctas_per_sm(kern, kQuantThreads, QuantSmem::bytes, cache[column_form ? 1 : 0]);
+    void (*kern)(const CUtensorMap, const MxParams) = !column_form ? quantize_mx_kernel<true, false>
+                                                      : row_form   ? quantize_mx_kernel<true, true>
+                                                                   : quantize_mx_kernel<false, true>;
+    static std::atomic<int> cache[3][64];   // row form, column form, both
+    const int which = row_form && column_form ? 2 : column_form ? 1 : 0;
+    const int per_sm = tile_ctas_per_sm(kern, kQuantThreads, QuantSmem::bytes, cache[which]);
     if (per_sm < 1) {
         const cudaError_t e = cudaGetLastError();
         return e != cudaSuccess ? e : cudaErrorInvalidValue;

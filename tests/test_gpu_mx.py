@@ -51,6 +51,42 @@ def test_mx_column_form(rows, cols, mode):
     _assert_mx_equal(g, codes, sw, f"MX column form {rows}x{cols} mode {mode}")
 
 
+# both forms from one read: each against the oracle, bit for bit; shapes with ragged 64-row and
+# 256-column tiles (multiples of 32 only, e.g. a last tile of 32 columns)
+@pytest.mark.parametrize("rows,cols", [(256, 256), (96, 160), (320, 544), (64, 1056), (1056, 96)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_mx_dual_forms(rows, cols, mode):
+    m = nv()
+    t = synth.grad_output(rows, cols, seed=5) if mode else synth.activations(rows, cols, seed=5, outlier_frac=0.02)
+    gr, gc = m.nvfp4_mx_quantize_dual(to_device_bf16(t), mode=mode, sr_seed=11, stream_row=1, stream_col=2)
+    bits = synth.bf16_bits(t)
+    codes, _, sw = _oracle_form(bits, 0, mode, 11, 1)
+    _assert_mx_equal(gr, codes, sw, f"MX dual, row form {rows}x{cols} mode {mode}")
+    codes, _, sw = _oracle_form(bits, 1, mode, 11, 2)
+    _assert_mx_equal(gc, codes, sw, f"MX dual, column form {rows}x{cols} mode {mode}")
+
+
+def test_mx_dual_full_size_equals_two_single_calls():
+    # the 8192 x 20480 gradient of the layer, SR: both forms equal the one-form calls'
+    m = nv()
+    g = torch.Generator(device="cpu").manual_seed(21)
+    x = (torch.randn((8192, 20480), generator=g) * 1e-2).to(torch.bfloat16).cuda()
+    gr, gc = m.nvfp4_mx_quantize_dual(x, mode=1, sr_seed=3, stream_row=1, stream_col=2)
+    r = m.nvfp4_mx_quantize(x, along=0, mode=1, sr_seed=3, stream_id=1)
+    c = m.nvfp4_mx_quantize(x, along=1, mode=1, sr_seed=3, stream_id=2)
+    torch.cuda.synchronize()
+    for a, b in ((gr, r), (gc, c)):
+        assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
+
+
+def test_mx_dual_shape_errors():
+    m = nv()
+    x = torch.zeros((48, 256), dtype=torch.bfloat16, device="cuda")   # rows % 32 != 0
+    with pytest.raises(m.NVFP4Error) as e:
+        m.nvfp4_mx_quantize_dual(x)
+    assert e.value.status == 3
+
+
 def test_mx_extreme_magnitudes():
     # scales at both ends of the UE8M0 range: huge, tiny (bf16 subnormal) and zero blocks
     m = nv()
