@@ -292,7 +292,6 @@ __device__ __forceinline__ U4 sr_words_p(const QuantParams& p, uint32_t stream_i
     return U4{c0, c1, c2, c3};
 }
 
-
 template <bool ROW, bool COL, bool SR>
 __global__ void __launch_bounds__(kQuantThreads, 3) quantize_tile_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                      const __grid_constant__ QuantParams p) {
