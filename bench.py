@@ -409,8 +409,9 @@ def run_ours(args, rank, world, local_rank):
                      "per_launch_flop": FLOP_GEMM, "avg_launch_ms": gemm_avg_ms},
         "quantize": {"gbs": q_gbs, "unit": "GB/s", "peak_hbm_gbs": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
                      "frac_of_8000_gbs": q_gbs / 8000.0,
-                     "bound": {"X": "instruction issue", "W": "instruction issue",
-                               "dY": "integer (ALU) pipe: Philox draws and the exact SR encode"},
+                     "bound": {"X": "instruction issue (64 % issue-active; ALU and FMA pipes ~50 %)",
+                               "W": "ALU pipe (61 %): 16x16 tile maxima and widening",
+                               "dY": "heavy FMA pipe (65 %: Philox products, f32x2 SR arithmetic) with the ALU (55 %)"},
                      "bytes_per_elem": Q_BYTES_PER_ELEM, "peak_basis": peak_kind,
                      "per_call_ms": {"X": statistics.mean(s_[0] for s_ in seg), "W": statistics.mean(s_[1] for s_ in seg),
                                      "dY": statistics.mean(s_[3] for s_ in seg)},

@@ -106,6 +106,20 @@ def test_nonfinite_is_flagged():
     assert m.nvfp4_poll(ws) == 0
 
 
+@pytest.mark.parametrize("bits", [0x7F80, 0xFF80, 0x7FC0, 0xFFC1])   # +inf, -inf, NaN, negative NaN
+@pytest.mark.parametrize("pos", [(0, 0), (5, 7), (31, 30), (16, 31)])  # both elements of a column pair
+def test_nonfinite_is_flagged_by_the_rht_amax_pass(bits, pos):
+    # the dual call's amax pass (plain amax as a NaN-propagating fp32 max, RHT amax alongside)
+    m = nv()
+    ws = m.Workspace()
+    x = torch.ones((32, 32), dtype=torch.bfloat16, device="cuda")
+    x.view(torch.int16)[pos] = bits - (1 << 16) if bits >= 1 << 15 else bits
+    m.nvfp4_quantize_dual(x, ws=ws)
+    assert m.nvfp4_poll(ws) == 7
+    m.nvfp4_quantize_dual(torch.ones((32, 32), dtype=torch.bfloat16, device="cuda"), ws=ws)
+    assert m.nvfp4_poll(ws) == 0
+
+
 def test_leading_dimension():
     m = nv()
     t, bits = _x(64, 256, seed=4)
