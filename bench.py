@@ -308,18 +308,23 @@ def run_ours(args, rank, world, local_rank):
 
         # Host-to-device copies, compute and device-to-host copies on three streams, ordered by
         # events so the two copy directions (PCIe is full duplex) overlap each other and the
-        # compute: step k's uploads wait for step k-1's compute to finish reading x, w and dy;
-        # its forward waits for x and w and for step k-1's read-back of y; its backward for dy
-        # and for step k-1's read-back of dx and dw; each read-back waits for its result.
+        # compute.  The inputs alternate between two device copies, so step k's uploads need
+        # only wait for step k-2's compute to finish reading its copy; step k's forward waits
+        # for its x and w and for step k-1's read-back of y; its backward for its dy and for
+        # step k-1's read-back of dx and dw; each read-back waits for its result.
         comp = torch.cuda.current_stream(dev)
         up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         evt = lambda: torch.cuda.Event()  # noqa: E731
-        prev = {"bwd": None, "y_read": None, "dxdw_read": None}
+        ins = [(x, w, dy), tuple(torch.empty_like(t) for t in (x, w, dy))]
+        prev = {"bwd": [None, None], "y_read": None, "dxdw_read": None, "k": 0}
 
         def e2e_step(seed):
+            slot = prev["k"] & 1
+            prev["k"] += 1
+            x, w, dy = ins[slot]
             with torch.cuda.stream(up_s):
-                if prev["bwd"] is not None:
-                    up_s.wait_event(prev["bwd"])
+                if prev["bwd"][slot] is not None:
+                    up_s.wait_event(prev["bwd"][slot])
                 x.copy_(hx, non_blocking=True)
                 w.copy_(hw, non_blocking=True)
                 xw_in = evt()
@@ -355,7 +360,8 @@ def run_ours(args, rank, world, local_rank):
                 hdw.copy_(dw_dev, non_blocking=True)
                 dxdw_read = evt()
                 dxdw_read.record(down_s)
-            prev.update(bwd=bwd_done, y_read=y_read, dxdw_read=dxdw_read)
+            prev["bwd"][slot] = bwd_done
+            prev.update(y_read=y_read, dxdw_read=dxdw_read)
 
         e2e_step(0)
         torch.cuda.synchronize()
@@ -378,7 +384,7 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "path": "pinned host X, W, dY -> nvfp4_linear_fwd/bwd (N > 1: the data-parallel step) -> pinned "
                        "host Y, dX, dW (N > 1: this rank's rows); uploads, compute and read-backs on three "
-                       "event-ordered streams"}
+                       "event-ordered streams, the inputs alternating between two device copies"}
 
     ffn = ffn_fields(args, world, dev, dist, flush) if args.ffn else None
     variants = variant_fields(args, dev, flush, x, w, dy) if args.variants else None
@@ -847,7 +853,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--workload", choices=["linear", "ffn"], default="linear",
                     help="linear: the 8192x5120x20480 layer (the default line); ffn: the one-FFN step")
